@@ -1,0 +1,501 @@
+#!/usr/bin/env python
+"""Throughput of the paged-KV attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one decode step of the Qwen3-0.6B-shaped layer (64 sequences,
+context U[128,4096], 16 q / 8 kv heads, head_dim 128, block_size 256):
+store_kvcache of the 64 new K/V rows, then paged GQA decode with split-KV and
+its merge pass.  Inputs are resident in HBM when the timed region starts;
+the KV working set (~0.55 GB) is larger than L2, so repeated steps read HBM.
+The headline value is decode KV bytes per second over all ranks.  The same
+JSON line carries the prefix-cached varlen prefill leg (32 sequences behind a
+shared 1024-token prefix) in TFLOP/s, the end-to-end number through host
+buffers, the roofline of the dominant kernel, and the oracle timed on the
+host cores.
+
+Under torchrun every rank runs its own independent batch (no collective on
+the data path); the timed region is bracketed by barriers and the reported
+time is the maximum over ranks.
+
+--impl reference times the CPU oracle (float64, OpenMP) on the same workload
+on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "decode KV bytes/s (% of HBM peak) and seqs/s; prefill TFLOP/s (% of peak)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+PROFILES = ROOT / "profiles"
+KERNEL_SOURCES = {
+    "decode": ["paged_kv_cache_331_b200/csrc/decode.cu", "paged_kv_cache_331_b200/csrc/pa_device.cuh"],
+    "prefill": ["paged_kv_cache_331_b200/csrc/prefill.cu", "paged_kv_cache_331_b200/csrc/pa_device.cuh"],
+}
+
+
+# ------------------------------------------------------------------------------------------ helpers --
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash(kind):
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kind]:
+        h.update((ROOT / f).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kind):
+    """DRAM bytes per launch recorded from an ncu capture, if the kernel source is unchanged since."""
+    for f in sorted(PROFILES.glob("*.md")) + sorted(PROFILES.glob("*.txt")):
+        text = f.read_text()
+        m = re.search(rf"traffic_per_launch\[{kind}\]\s*=\s*([0-9.eE+]+)\s+source_sha=([0-9a-f]+)", text)
+        if m:
+            return float(m.group(1)) if m.group(2) == kernel_source_hash(kind) else None
+    return None
+
+
+def decode_algorithmic_bytes(w):
+    """Bytes the decode step must move: every in-context K and V row once per kv head, q, out, tables."""
+    L = w.context_lens.astype(np.int64)
+    kv = int(L.sum()) * w.num_kv_heads * w.head_dim * 2 * 2
+    qo = 2 * w.num_seqs * w.num_heads * w.head_dim * 2
+    tables = int(np.ceil(L / w.block_size).sum()) * 4 + w.num_seqs * 4
+    return kv, kv + qo + tables
+
+
+def prefill_flops(w):
+    """4 * D * Hq per unmasked (query, key) pair: QK^T and PV, each a multiply-add."""
+    total = 0
+    for b in range(w.num_seqs):
+        lq = int(w.cu_seqlens_q[b + 1] - w.cu_seqlens_q[b]); lk = int(w.cu_seqlens_k[b + 1] - w.cu_seqlens_k[b])
+        if w.causal:
+            total += lq * (lk - lq) + lq * (lq + 1) // 2
+        else:
+            total += lq * lk
+    return 4 * w.head_dim * w.num_heads * total
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons while the timed region runs (NVML, nvidia-smi fallback)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, torch_device_index, period_s=0.005):
+        self.samples, self.max_mhz, self.err = [], None, None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            idx = torch_device_index
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                ids = [v.strip() for v in vis.split(",") if v.strip()]
+                if torch_device_index < len(ids) and ids[torch_device_index].isdigit():
+                    idx = int(ids[torch_device_index])
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nvml = pynvml
+        except Exception as e:  # noqa: BLE001
+            self.err = f"nvml: {e}"
+
+    def _reasons(self):
+        p = self._nvml
+        fn = getattr(p, "nvmlDeviceGetCurrentClocksEventReasons", None) or p.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self._h)
+
+    def _run(self):
+        p = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append((p.nvmlDeviceGetClockInfo(self._h, p.NVML_CLOCK_SM),
+                                     p.nvmlDeviceGetPowerUsage(self._h) / 1000.0, int(self._reasons())))
+            except Exception as e:  # noqa: BLE001
+                self.err = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": self.err or "no samples"}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[2]
+        reasons = sorted(name for bit, name in self.REASONS.items() if bits & bit)
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "power_w_max": round(max(s[1] for s in self.samples), 1)}
+
+
+# ---------------------------------------------------------------------------------------- distributed --
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif args.impl == "ours":
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# -------------------------------------------------------------------------------------------- ours --
+
+def to_dev(a, kind, dev):
+    import torch
+    if kind == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+
+
+def pinned(a, kind):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if kind == "bf16"
+                         else np.ascontiguousarray(a, dtype=np.int32))
+    t = t.view(torch.bfloat16) if kind == "bf16" else t
+    return t.pin_memory()
+
+
+def bench_decode(args, world, rank, dev, peaks):
+    import torch
+    import paged_kv_cache_331_b200 as pa
+    from paged_kv_cache_331_b200 import workloads as W
+
+    w = W.qwen3_decode(seed=2 + 1000 * rank)
+    q, kc, vc = to_dev(w.q, "bf16", dev), to_dev(w.k_cache, "bf16", dev), to_dev(w.v_cache, "bf16", dev)
+    nk, nv = to_dev(w.new_k, "bf16", dev), to_dev(w.new_v, "bf16", dev)
+    slots, bt, cl = to_dev(w.slot_mapping, "i32", dev), to_dev(w.block_tables, "i32", dev), to_dev(w.context_lens, "i32", dev)
+    out = torch.empty_like(q)
+    maxL = w.max_context_len
+    ws_bytes = pa.decode_workspace_size(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, maxL, w.block_size, 0)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    chunk = pa.decode_chunk_size(w.num_seqs, w.num_kv_heads, maxL, w.block_size)
+    launches_per_step = 2 + (1 if ws_bytes > 0 else 0)
+
+    def step():
+        pa.store_kvcache(nk, nv, kc, vc, slots)
+        pa.decode(q, kc, vc, bt, cl, maxL, w.scale, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        t0.record()
+        for i in range(K):
+            ev[i][0].record()
+            pa.store_kvcache(nk, nv, kc, vc, slots)
+            ev[i][1].record()
+            pa.decode(q, kc, vc, bt, cl, maxL, w.scale, out=out, workspace=ws)
+            ev[i][2].record()
+        t1.record()
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    elapsed_ms = t0.elapsed_time(t1)
+    store_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    decode_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    assert pa.device_error() == 0
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+
+    kv_bytes, alg_bytes = decode_algorithmic_bytes(w)
+    total_kv = sum_over_ranks(float(kv_bytes), world) * K
+    value = total_kv / (elapsed_ms / 1e3) / 1e9
+    seqs = sum_over_ranks(float(w.num_seqs), world) * K / (elapsed_ms / 1e3)
+    achieved = alg_bytes / (decode_ms / 1e3) / 1e9
+    traffic = profiled_traffic("decode")
+
+    # end to end through host buffers: per step H2D of q, new K/V rows and the metadata, D2H of out
+    hq_, hnk, hnv = pinned(w.q, "bf16"), pinned(w.new_k, "bf16"), pinned(w.new_v, "bf16")
+    hs, hbt, hcl = pinned(w.slot_mapping, "i32"), pinned(w.block_tables, "i32"), pinned(w.context_lens, "i32")
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq_, hnk, hnv, hs, hbt, hcl))
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        q.copy_(hq_, non_blocking=True); nk.copy_(hnk, non_blocking=True); nv.copy_(hnv, non_blocking=True)
+        slots.copy_(hs, non_blocking=True); bt.copy_(hbt, non_blocking=True); cl.copy_(hcl, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+
+    for _ in range(min(args.warmup, 10)):
+        e2e_step()
+    Ke = max(1, min(K, 500))
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(Ke):
+        e2e_step()
+    s1.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
+    e2e_value = sum_over_ranks(float(kv_bytes), world) * Ke / (e2e_ms / 1e3) / 1e9
+
+    return w, {
+        "value": value, "ms_per_step": elapsed_ms / K, "seqs_per_s": seqs, "store_ms": store_ms,
+        "decode_ms": decode_ms, "kv_bytes_per_step": kv_bytes, "alg_bytes": alg_bytes, "achieved": achieved,
+        "traffic": traffic, "chunk": chunk, "ws_bytes": ws_bytes, "launches": launches_per_step * K,
+        "clocks": clk.summary(), "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                                         "d2h_bytes_per_step": d2h, "steps": Ke},
+    }
+
+
+def bench_prefill(args, dev, peaks):
+    import torch
+    import paged_kv_cache_331_b200 as pa
+    from paged_kv_cache_331_b200 import workloads as W
+
+    w = W.prefix_prefill()
+    q, kc, vc = to_dev(w.q, "bf16", dev), to_dev(w.k_cache, "bf16", dev), to_dev(w.v_cache, "bf16", dev)
+    nk, nv = to_dev(w.new_k, "bf16", dev), to_dev(w.new_v, "bf16", dev)
+    slots, bt = to_dev(w.slot_mapping, "i32", dev), to_dev(w.block_tables, "i32", dev)
+    cq, ck = to_dev(w.cu_seqlens_q, "i32", dev), to_dev(w.cu_seqlens_k, "i32", dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2, written between reps
+
+    def store():
+        pa.store_kvcache(nk, nv, kc, vc, slots)
+
+    def prefill():
+        pa.prefill_varlen(q, kc, vc, cq, ck, w.max_seqlen_q, w.max_seqlen_k, bt, w.scale, True, out=out)
+
+    for _ in range(max(3, min(args.warmup, 10))):
+        store(); prefill()
+    torch.cuda.synchronize(dev)
+    reps = max(3, min(args.steps, 100))
+    st, pf = [], []
+    for _ in range(reps):
+        flush.zero_()
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(); store(); b.record(); prefill(); c.record()
+        st.append((a, b)); pf.append((b, c))
+    torch.cuda.synchronize(dev)
+    store_ms = float(np.median([x.elapsed_time(y) for x, y in st]))
+    prefill_ms = float(np.median([x.elapsed_time(y) for x, y in pf]))
+    assert pa.device_error() == 0
+    flops = prefill_flops(w)
+    tflops = flops / (prefill_ms / 1e3) / 1e12
+    store_bytes = 2 * 2 * int(w.cu_seqlens_q[-1]) * w.num_kv_heads * w.head_dim * 2 + 4 * int(w.cu_seqlens_q[-1])
+    store_gbs = store_bytes / (store_ms / 1e3) / 1e9
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    return {
+        "workload": w.name, "num_seqs": w.num_seqs, "prefix_len": 1024, "suffix": "U[64,512]",
+        "total_q": int(w.cu_seqlens_q[-1]), "ms": prefill_ms, "flops": flops, "tflops": tflops,
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": tflops / peak_tf, "traffic": profiled_traffic("prefill"),
+                     "peak_kind": f"bf16 burst ({peaks.get('source')})"},
+        "store": {"rows": int(w.cu_seqlens_q[-1]), "ms": store_ms, "gbs": store_gbs,
+                  "frac": store_gbs / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "bytes": store_bytes},
+        "gpu_launches_per_rep": 2,
+    }
+
+
+def cpu_baseline(w, budget_s=12.0):
+    """The oracle as it stands, on this host's cores: store + decode of the same workload, repeated for about
+    budget_s seconds."""
+    from oracle import oracle as O
+    orc = O.get()
+    kc, vc = w.k_cache.copy(), w.v_cache.copy()
+    kv_bytes, _ = decode_algorithmic_bytes(w)
+    reps, t_total = 0, 0.0
+    while t_total < budget_s and reps < 50:
+        t = time.perf_counter()
+        orc.store_kvcache(w.new_k, w.new_v, kc, vc, w.slot_mapping)
+        orc.decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale)
+        t_total += time.perf_counter() - t
+        reps += 1
+    return {"value": kv_bytes * reps / t_total / 1e9, "unit": "GB/s", "cores": orc.max_threads(), "kind": "oracle",
+            "sample": f"full workload (store + decode of all {w.num_seqs} sequences), {reps} rep(s), "
+                      f"{t_total:.1f} s", "seconds": t_total}
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    peaks = load_peaks()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    import paged_kv_cache_331_b200 as pa
+    pa.lib()
+    w, d = bench_decode(args, world, rank, dev, peaks)
+    pre = bench_prefill(args, dev, peaks) if (rank == 0 and not args.no_prefill) else None
+    cpu = cpu_baseline(w) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if rank != 0:
+        return
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    line = {
+        "metric": METRIC, "value": round(d["value"], 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(d["ms_per_step"], 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32",
+        "data": "synthetic: seeded N(0,1) bf16 Q/K/V, block tables drawn from a shuffled 1.25x pool",
+        "config": {"workload": w.name, "num_seqs": w.num_seqs, "context_lens": "U[128,4096]",
+                   "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "pool_blocks": w.num_blocks, "kv_bytes_per_step": d["kv_bytes_per_step"],
+                   "step": "store_kvcache(64 rows) + decode (split-KV + merge)", "kv_chunk_size": d["chunk"],
+                   "l2": f"inputs larger than L2: {d['kv_bytes_per_step'] / 1e6:.0f} MB KV per step vs 126 MB L2",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "seqs_per_s": round(d["seqs_per_s"], 1),
+        "hbm_frac": round(d["value"] / world / hbm, 4),
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_split_kernel + merge)",
+                     "achieved": round(d["achieved"], 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(d["achieved"] / hbm, 4), "traffic": d["traffic"],
+                     "algorithmic_bytes": d["alg_bytes"], "launch_ms": round(d["decode_ms"], 5),
+                     "peak_kind": f"HBM copy ({peaks.get('source')})"},
+        "store": {"ms": round(d["store_ms"], 5), "rows": w.num_seqs},
+        "e2e": d["e2e"], "gpu_launches": d["launches"], "clocks": d["clocks"],
+    }
+    if pre is not None:
+        line["prefill"] = pre
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------------------- reference --
+
+def run_reference(args, world, rank):
+    """The CPU oracle on the host cores, each step a bounded sample of the same workload."""
+    if rank != 0:
+        return
+    from oracle import oracle as O
+    from paged_kv_cache_331_b200 import workloads as W
+    orc = O.get()
+    w = W.qwen3_decode()
+    # calibrate: sequences per step so that warmup + steps end within about two minutes
+    one = W.decode_workload(w.context_lens[:1], w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                            rng=np.random.default_rng(0))
+    t = time.perf_counter()
+    orc.decode(one.q, one.k_cache, one.v_cache, one.block_tables, one.context_lens, one.scale)
+    t1 = max(time.perf_counter() - t, 1e-4) * max(1.0, 2112.0 / float(one.context_lens[0]))
+    per_step_budget = 120.0 / max(1, args.steps + args.warmup)
+    nseq = int(max(1, min(w.num_seqs, per_step_budget / t1)))
+    sub = slice(0, nseq)
+    kc, vc = w.k_cache.copy(), w.v_cache.copy()
+
+    def step():
+        orc.store_kvcache(w.new_k[sub], w.new_v[sub], kc, vc, w.slot_mapping[sub])
+        orc.decode(w.q[sub], kc, vc, w.block_tables[sub], w.context_lens[sub], w.scale)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t
+    kv = int(w.context_lens[sub].astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 4
+    value = kv * args.steps / el / 1e9
+    sample = f"first {nseq} of {w.num_seqs} sequences per step (store + decode)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded N(0,1) bf16 Q/K/V, block tables drawn from a shuffled 1.25x pool",
+        "config": {"workload": w.name, "num_seqs": w.num_seqs, "context_lens": "U[128,4096]",
+                   "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": orc.max_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

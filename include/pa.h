@@ -1,0 +1,188 @@
+/*
+ * pa.h -- C ABI of the paged-KV attention library (libpagedattn.so), sm_100a.
+ *
+ * The library implements the attention step of a nano-vLLM-style serving
+ * engine over a paged KV cache:
+ *
+ *   pa_store_kvcache   scatter the new tokens' K/V rows into cache slots
+ *   pa_decode          one query token per sequence against its cached keys
+ *                      (GQA; long contexts split across CTAs + a merge pass)
+ *   pa_prefill_varlen  causal varlen prefill whose leading blocks may be
+ *                      shared prefix-cache blocks
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * - Pointers named *_cache, q, out, key, value, block_tables, context_lens,
+ *   cu_seqlens_*, slot_mapping and workspace are DEVICE pointers owned by the
+ *   caller.  The library never allocates, frees or retains them.
+ * - bf16 tensors are passed as void*; their layouts are stated per argument.
+ *   Every tensor is dense row-major unless a row stride is given.
+ * - k_cache / v_cache are one layer's cache, [num_blocks, block_size,
+ *   num_kv_heads, head_dim] bf16 ("Architektur im Überblick", section
+ *   "Dynamische KV-Cache-Allokation": the per-layer views of the engine's
+ *   [2, num_layers, num_blocks, block_size, kv_heads, head_dim] tensor).
+ *   Base addresses must be 16-byte aligned.
+ * - stream is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *   asynchronous on that stream; none synchronises the host.
+ * - Argument and shape errors are reported synchronously, before anything is
+ *   launched: PA_ERR_INVALID_ARG for values outside the contract,
+ *   PA_ERR_UNSUPPORTED for legal shapes this build has no kernel for,
+ *   PA_ERR_WORKSPACE for a workspace that is too small, PA_ERR_CUDA when a
+ *   launch fails (pa_last_error() then holds the CUDA message).
+ * - Device-side contract (not checked on the device): block ids in the used
+ *   part of block_tables lie in [0, num_blocks); slots are unique;
+ *   context_lens[b] <= max_context_len and <= max_blocks_per_seq*block_size.
+ * - Supported: head_dim 64 or 128; num_heads a multiple of num_kv_heads
+ *   with group size G = num_heads / num_kv_heads in 1..8 for decode and
+ *   G in {1, 2, 4, 8} for prefill; block_size a power of two in [16, 1024];
+ *   num_blocks * block_size < 2^31.
+ */
+#ifndef PAGED_ATTN_PA_H
+#define PAGED_ATTN_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,
+    PA_ERR_UNSUPPORTED = 2,
+    PA_ERR_CUDA = 3,
+    PA_ERR_WORKSPACE = 4
+} pa_status;
+
+/* Static string naming a status code. */
+PA_API const char* pa_status_string(int status);
+
+/* Message describing the last failed call on this host thread ("" if none). */
+PA_API const char* pa_last_error(void);
+
+/* Library ABI version: (major << 16) | minor. */
+PA_API int32_t pa_version(void);
+
+/*
+ * pa_store_kvcache -- write the new tokens' K/V rows into the cache.
+ * ("Nano-vLLM 源碼學習" §二.2: a store_kvcache kernel stores key and value
+ * into the cache; "Architektur im Überblick", "Prefill- und
+ * Decode-Vorbereitung": the engine builds one slot per new token.)
+ *
+ * For each t in [0, num_tokens) with s = slot_mapping[t] != -1:
+ *   k_cache[s / block_size][s % block_size][:][:] = key[t][:][:]
+ *   v_cache[s / block_size][s % block_size][:][:] = value[t][:][:]
+ * A bit copy.  Slots equal to -1 are skipped; a slot outside
+ * [0, num_blocks*block_size) other than -1 breaks the contract and is also
+ * skipped, never written out of bounds.
+ *
+ * key, value:    [num_tokens, num_kv_heads, head_dim] bf16, row t starting at
+ *                element t*key_row_stride (t*value_row_stride); the strides
+ *                are in elements and may exceed num_kv_heads*head_dim (views
+ *                into a fused QKV buffer).
+ * slot_mapping:  [num_tokens] int32.
+ * num_tokens == 0 launches nothing and returns PA_OK.
+ */
+PA_API pa_status pa_store_kvcache(const void* key, const void* value, int64_t key_row_stride, int64_t value_row_stride,
+                           void* k_cache, void* v_cache, const int32_t* slot_mapping, int32_t num_tokens,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                           void* stream);
+
+/*
+ * pa_decode_chunk_size -- tokens per split-KV chunk that pa_decode uses when
+ * its kv_chunk_size argument is 0, for this shape on the current device.
+ * Returns a multiple of 64, or a value >= max_context_len meaning "no split";
+ * returns -1 for invalid arguments.
+ */
+PA_API int32_t pa_decode_chunk_size(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int32_t block_size);
+
+/*
+ * pa_decode_workspace_size -- bytes of workspace pa_decode needs for these
+ * arguments (0 when no sequence is split).  kv_chunk_size as for pa_decode.
+ * Returns 0 for invalid arguments as well; pa_decode then reports them.
+ */
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t block_size, int32_t kv_chunk_size);
+
+/*
+ * pa_decode -- paged GQA decode, one query token per sequence.
+ * ("Nano-vLLM 源碼學習" §二.2, decode stage: attention against the KV cache;
+ * lshu.cn essay on Nano-vLLM §3.2: K/V of logical position j of a sequence
+ * are gathered from page j / block_size, offset j % block_size of its page
+ * table.)
+ *
+ * For b in [0, num_seqs), h in [0, num_heads), L = context_lens[b],
+ * g = h / (num_heads / num_kv_heads), K_j = k_cache[block_tables[b][j/bs]][j%bs][g]:
+ *   out[b][h] = sum_{j<L} softmax_j(scale * <q[b][h], K_j>) * V_j
+ * L == 0 gives out[b][h] = 0.  The newest token (position L-1) must already
+ * be in the cache (call pa_store_kvcache first).
+ *
+ * q, out:         [num_seqs, num_heads, head_dim] bf16 (dense).
+ * block_tables:   [num_seqs, max_blocks_per_seq] int32; entries past
+ *                 ceil(L/block_size) are never read (may be -1).
+ * context_lens:   [num_seqs] int32, each <= max_context_len.
+ * kv_chunk_size:  0 = automatic; otherwise tokens per split-KV chunk, a
+ *                 multiple of 64 (a value >= max_context_len disables the
+ *                 split).  Sequences longer than one chunk are processed by
+ *                 several CTAs whose partial (max, sum, weighted V) results
+ *                 are merged by a second kernel.
+ * workspace:      device buffer of at least pa_decode_workspace_size(...)
+ *                 bytes (may be NULL when that size is 0); fully written
+ *                 before it is read, so its contents need no initialisation.
+ *                 Concurrent calls must not share a workspace.
+ */
+PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                    int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t kv_chunk_size,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * pa_prefill_varlen -- varlen causal prefill against the paged cache.
+ * ("Nano-vLLM 源碼學習" §二.2, prefill stage: varlen attention with prefix
+ * cache support; "Architektur im Überblick", "Prefill- und
+ * Decode-Vorbereitung": only the uncached tokens are computed and their
+ * positions start at num_cached_tokens; "Hash-basiertes Prefix Caching":
+ * cached prefix blocks are whole blocks shared by reference.)
+ *
+ * Sequence b has Lq = cu_seqlens_q[b+1]-cu_seqlens_q[b] query tokens (its
+ * uncached tokens, whose K/V were stored with pa_store_kvcache beforehand)
+ * and Lk = cu_seqlens_k[b+1]-cu_seqlens_k[b] >= Lq keys, all read from the
+ * cache through block_tables[b].  Query i sits at position Lk - Lq + i; with
+ * causal != 0 it attends keys 0 .. Lk-Lq+i, otherwise keys 0 .. Lk-1.
+ *
+ * q, out:         [total_q, num_heads, head_dim] bf16 (dense), total_q =
+ *                 cu_seqlens_q[num_seqs] - cu_seqlens_q[0]; row t of q/out
+ *                 belongs to the sequence b with cu_seqlens_q[b] <= t +
+ *                 cu_seqlens_q[0] < cu_seqlens_q[b+1].
+ * cu_seqlens_q/k: [num_seqs+1] int32, non-decreasing.
+ * max_seqlen_q/k: upper bounds of Lq and Lk over the batch.
+ * block_tables:   as for pa_decode, entries past ceil(Lk/block_size) unread.
+ */
+PA_API pa_status pa_prefill_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t total_q,
+                            int32_t max_seqlen_q, int32_t max_seqlen_k, const int32_t* block_tables,
+                            int32_t max_blocks_per_seq, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                            int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t causal,
+                            void* stream);
+
+/*
+ * pa_device_error -- read and clear the library's device-side error word on
+ * the current device (synchronises the given stream).  Kernels set it instead
+ * of hanging when a pipeline wait exceeds its time limit (about one second);
+ * 0 means no error.  Diagnostic only.
+ */
+PA_API pa_status pa_device_error(int32_t* code_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_ATTN_PA_H */

@@ -1,0 +1,18 @@
+"""Attention over a paged KV cache on B200 (sm_100a).
+
+The computation lives in ``libpagedattn.so`` (C ABI in ``include/pa.h``);
+this package is its Python face:
+
+    store_kvcache(key, value, k_cache, v_cache, slot_mapping)
+    decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale)
+    prefill_varlen(q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                   block_tables, scale, causal=True)
+
+The shared library is loaded on first use; importing the package does not
+touch CUDA.  ``workloads`` builds seeded synthetic inputs.
+"""
+from ._binding import (PagedAttentionError, decode, decode_chunk_size, decode_workspace_size, device_error, lib,
+                       prefill_varlen, store_kvcache)
+
+__all__ = ["store_kvcache", "decode", "prefill_varlen", "decode_workspace_size", "decode_chunk_size", "device_error",
+           "PagedAttentionError", "lib"]

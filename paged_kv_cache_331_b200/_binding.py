@@ -1,0 +1,163 @@
+"""ctypes binding of libpagedattn.so (the C ABI declared in include/pa.h).
+
+Argument marshalling only: torch tensors supply device pointers, shapes and
+the current CUDA stream; every step of the computation runs in the library's
+kernels.  There is no fallback: if the library is missing or the tensors are
+not CUDA tensors, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+LIB_PATH = Path(__file__).resolve().parent / "libpagedattn.so"
+
+PA_OK = 0
+_lib = None
+
+_i32, _i64, _f32, _sz, _vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+
+_PROTOS = {
+    "pa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "pa_last_error": (ctypes.c_char_p, []),
+    "pa_version": (_i32, []),
+    "pa_store_kvcache": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "pa_decode_chunk_size": (_i32, [_i32, _i32, _i32, _i32]),
+    "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    "pa_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
+                                 _i32, _vp, _sz, _vp]),
+    "pa_prefill_varlen": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _i32, _i32, _i32,
+                                         _i32, _i32, _i32, _f32, _i32, _vp]),
+    "pa_device_error": (ctypes.c_int, [ctypes.POINTER(_i32), _vp]),
+}
+
+
+class PagedAttentionError(RuntimeError):
+    pass
+
+
+def lib() -> ctypes.CDLL:
+    """Load libpagedattn.so once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise ImportError(f"{LIB_PATH.name} is missing; build it with `python -m paged_kv_cache_331_b200.build`")
+        L = ctypes.CDLL(str(LIB_PATH))
+        for name, (res, args) in _PROTOS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != PA_OK:
+        L = lib()
+        raise PagedAttentionError(f"{what}: {L.pa_status_string(status).decode()}: {L.pa_last_error().decode()}")
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _dense(t: torch.Tensor, name: str) -> None:
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(t: torch.Tensor, stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(t.device)
+    return s.cuda_stream
+
+
+def store_kvcache(key, value, k_cache, v_cache, slot_mapping, stream=None) -> None:
+    """Scatter key/value rows [N, Hkv, D] into k_cache/v_cache at slot_mapping (-1 = skip)."""
+    for n, t in (("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _cuda(t, n, torch.bfloat16)
+    _cuda(slot_mapping, "slot_mapping", torch.int32)
+    _dense(k_cache, "k_cache"); _dense(v_cache, "v_cache"); _dense(slot_mapping, "slot_mapping")
+    nb, bs, hkv, d = k_cache.shape
+    n = slot_mapping.shape[0]
+    for name, t in (("key", key), ("value", value)):
+        if t.shape[0] != n or tuple(t.shape[1:]) != (hkv, d) or t.stride(-1) != 1 or t.stride(-2) != d:
+            raise ValueError(f"{name} must be [N, {hkv}, {d}] with dense rows")
+    with torch.cuda.device(k_cache.device):
+        _check(lib().pa_store_kvcache(key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0),
+                                      k_cache.data_ptr(), v_cache.data_ptr(), slot_mapping.data_ptr(), n, hkv, d, bs,
+                                      nb, _stream(k_cache, stream)), "pa_store_kvcache")
+
+
+def decode_chunk_size(num_seqs, num_kv_heads, max_context_len, block_size) -> int:
+    return int(lib().pa_decode_chunk_size(num_seqs, num_kv_heads, max_context_len, block_size))
+
+
+def decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, block_size,
+                          kv_chunk_size=0) -> int:
+    return int(lib().pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                                              block_size, kv_chunk_size))
+
+
+def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, *, out=None, workspace=None,
+           kv_chunk_size=0, stream=None):
+    """Paged GQA decode: q [B, Hq, D] -> out [B, Hq, D]."""
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _cuda(t, n, torch.bfloat16); _dense(t, n)
+    _cuda(block_tables, "block_tables", torch.int32); _dense(block_tables, "block_tables")
+    _cuda(context_lens, "context_lens", torch.int32); _dense(context_lens, "context_lens")
+    B, hq, d = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    if d2 != d:
+        raise ValueError("head_dim of q and the cache differ")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _cuda(out, "out", torch.bfloat16); _dense(out, "out")
+    need = decode_workspace_size(B, hq, hkv, d, int(max_context_len), bs, kv_chunk_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(q.device):
+        _check(lib().pa_decode(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                               block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+                               int(max_context_len), B, hq, hkv, d, bs, nb, float(scale), int(kv_chunk_size), ws_ptr,
+                               ws_len, _stream(q, stream)), "pa_decode")
+    return out
+
+
+def prefill_varlen(q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, block_tables, scale,
+                   causal=True, *, out=None, stream=None):
+    """Varlen prefill over the paged cache: q [total_q, Hq, D] -> out [total_q, Hq, D]."""
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _cuda(t, n, torch.bfloat16); _dense(t, n)
+    for n, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k), ("block_tables", block_tables)):
+        _cuda(t, n, torch.int32); _dense(t, n)
+    total_q, hq, d = q.shape
+    nb, bs, hkv, _ = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _cuda(out, "out", torch.bfloat16); _dense(out, "out")
+    with torch.cuda.device(q.device):
+        _check(lib().pa_prefill_varlen(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                       cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), total_q, int(max_seqlen_q),
+                                       int(max_seqlen_k), block_tables.data_ptr(), block_tables.shape[1],
+                                       cu_seqlens_q.shape[0] - 1, hq, hkv, d, bs, nb, float(scale), int(bool(causal)),
+                                       _stream(q, stream)), "pa_prefill_varlen")
+    return out
+
+
+def device_error(stream=None, device=None) -> int:
+    """Read and clear the library's device-side error word (synchronises the stream)."""
+    dev = device if device is not None else torch.cuda.current_device()
+    code = _i32(0)
+    with torch.cuda.device(dev):
+        s = stream.cuda_stream if stream is not None else torch.cuda.current_stream(dev).cuda_stream
+        _check(lib().pa_device_error(ctypes.byref(code), s), "pa_device_error")
+    return int(code.value)

@@ -1,0 +1,461 @@
+// Paged GQA decode with split-KV, for sm_100a.
+//
+// ("Nano-vLLM 源碼學習" §二.2, decode stage; the lshu.cn essay on Nano-vLLM
+// §3.2: attention gathers K/V of position j from page j / block_size, offset
+// j % block_size of the sequence's page table.)
+//
+// The decode step reads every cached K/V row of every sequence once and does
+// 4*G*D flops per row pair (G = query heads per kv head): about 2-4 flops per
+// byte, so it is bound by HBM bandwidth, not by arithmetic.  Design:
+//
+//  * One CTA per (chunk of a sequence's keys, kv head, sequence).  The CTA
+//    handles all G query heads that share the kv head, so each K/V byte
+//    crosses HBM once.  Long sequences are cut into several chunks; their
+//    partial results (running max m, sum l, unnormalised weighted V) go to a
+//    workspace and a second kernel merges them (log-sum-exp rescaling).
+//  * A producer warp streams 64-token K and V tiles of the kv head into
+//    shared memory with TMA (a 3-D tensor map over [num_blocks*block_size,
+//    kv_heads, head_dim] makes the physical block id just a row
+//    coordinate), kStages deep, signalled through mbarriers.
+//  * Four consumer warps each own 16 tokens of a tile.  QK: 8 lanes per
+//    token, each lane holding D/8 query elements per head in registers,
+//    three xor-shuffles per head finish the dot product.  Online softmax in
+//    the exp2 domain (q pre-scaled by scale*log2 e) per warp.  PV: each lane
+//    owns D/32 output dims of every head and walks the warp's tokens, reading
+//    the probabilities as a shared-memory broadcast.  Warps merge their
+//    (m, l, acc) at the end through shared memory.
+#include <cuda_runtime.h>
+
+#include <math.h>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr int kTile = kDecodeTile;         // tokens per stage
+constexpr int kWarps = 4;                  // consumer warps
+constexpr int kTPW = kTile / kWarps;       // tokens per consumer warp per tile
+constexpr int kRounds = kTPW / 4;          // QK rounds (4 tokens per warp per round)
+constexpr int kStages = 4;
+constexpr int kThreads = (kWarps + 1) * 32;
+
+struct DecodeParams {
+  __nv_bfloat16* out;
+  const __nv_bfloat16* q;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* ws_acc;
+  float* ws_ml;
+  int32_t max_blocks_per_seq;
+  int32_t max_context_len;
+  int32_t num_heads;
+  int32_t block_size;
+  int32_t box_rows;
+  int32_t chunk_tokens;
+  int32_t max_chunks;
+  float scale_log2;
+  unsigned int* err;
+};
+
+template <int D, int G>
+struct DecodeSmem {
+  static constexpr size_t kv_stage_elems = static_cast<size_t>(kTile) * D;
+  static constexpr size_t k_off = 0;
+  static constexpr size_t v_off = k_off + kStages * kv_stage_elems * 2;
+  static constexpr size_t p_off = v_off + kStages * kv_stage_elems * 2;
+  static constexpr size_t m_off = p_off + static_cast<size_t>(kWarps) * kTPW * G * 4;
+  static constexpr size_t bar_off = m_off + static_cast<size_t>(kWarps) * G * (D + 2) * 4;
+  static constexpr size_t bytes = bar_off + 2 * kStages * 8;
+  static_assert(m_off % 8 == 0 && bar_off % 8 == 0, "alignment");
+};
+
+__device__ __forceinline__ int clamp_context(int L, const DecodeParams& p) {
+  L = min(L, p.max_context_len);
+  L = min(L, p.max_blocks_per_seq * p.block_size);
+  return max(L, 0);
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const DecodeParams p) {
+  using Smem = DecodeSmem<D, G>;
+  constexpr int DPL = D / 8;    // query/key dims per lane in QK (8 lanes per token)
+  constexpr int DPV = D / 32;   // output dims per lane in PV
+  static_assert(D == 64 || D == 128, "head_dim");
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + Smem::k_off);
+  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + Smem::v_off);
+  float* pbuf = reinterpret_cast<float*>(smem + Smem::p_off);
+  float* mrg = reinterpret_cast<float*>(smem + Smem::m_off);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Smem::bar_off);
+  uint64_t* empty = full + kStages;
+
+  const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int L = clamp_context(__ldg(p.context_lens + b), p);
+  const int hq0 = g * G;
+
+  if (L == 0) {   // no keys: the output is defined as zero
+    if (chunk == 0)
+      for (int i = threadIdx.x; i < G * D; i += kThreads)
+        p.out[(static_cast<int64_t>(b) * p.num_heads + hq0) * D + i] = __float2bfloat16(0.f);
+    return;
+  }
+  const int start = chunk * p.chunk_tokens;
+  if (start >= L) return;
+  const int end = min(L, start + p.chunk_tokens);
+  const int nchunks = (L + p.chunk_tokens - 1) / p.chunk_tokens;
+  const int ntiles = (end - start + kTile - 1) / kTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kWarps) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+      const uint64_t pol = policy_evict_first();
+      const int bs_shift = __ffs(p.block_size) - 1;
+      int issued = 0;
+      for (int it = 0; it < ntiles; ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, p.err)) break;
+        const int t0 = start + it * kTile;
+        const int valid = min(kTile, end - t0);
+        const int nbox = (valid + p.box_rows - 1) / p.box_rows;
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * p.box_rows * D * 2 * 2));
+        for (int k = 0; k < nbox; ++k) {
+          const int tok = t0 + k * p.box_rows;
+          const int blk = __ldg(bt + (tok >> bs_shift));
+          const int row = (blk << bs_shift) + (tok & (p.block_size - 1));
+          const size_t soff = (static_cast<size_t>(s) * kTile + static_cast<size_t>(k) * p.box_rows) * D;
+          tma_load_3d_hint(sK + soff, &tmK, &full[s], 0, g, row, pol);
+          tma_load_3d_hint(sV + soff, &tmV, &full[s], 0, g, row, pol);
+        }
+        ++issued;
+      }
+      // Never leave with copies in flight: wait (time-limited) for the last
+      // loads of every stage.  On the normal path these have long landed.
+      for (int it = max(0, issued - kStages); it < issued; ++it)
+        mbar_wait(&full[it % kStages], (it / kStages) & 1, p.err, kErrDrainTimeout);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers --
+  const int li = lane & 7, gi = lane >> 3;
+  float qf[G][DPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const __nv_bfloat16* qp = p.q + (static_cast<int64_t>(b) * p.num_heads + hq0 + h) * D;
+#pragma unroll
+    for (int part = 0; part < DPL / 8; ++part) {
+      const uint4 v = *reinterpret_cast<const uint4*>(qp + part * 64 + li * 8);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qf[h][part * 8 + 2 * e] = bf16lo(w[e]) * p.scale_log2;
+        qf[h][part * 8 + 2 * e + 1] = bf16hi(w[e]) * p.scale_log2;
+      }
+    }
+  }
+  float m[G], l[G], acc[G][DPV];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+#pragma unroll
+    for (int c = 0; c < DPV; ++c) acc[h][c] = 0.f;
+  }
+  float* pw = pbuf + warp * kTPW * G;
+  const int wbase = warp * kTPW;
+
+  for (int it = 0; it < ntiles; ++it) {
+    const int s = it % kStages;
+    if (!mbar_wait(&full[s], (it / kStages) & 1, p.err)) break;
+    const int valid = min(kTile, end - (start + it * kTile));
+    const int nw = min(kTPW, valid - wbase);
+    if (nw > 0) {
+      const __nv_bfloat16* Ks = sK + static_cast<size_t>(s) * kTile * D;
+      float sc[kRounds][G];
+#pragma unroll
+      for (int r = 0; r < kRounds; ++r) {
+        const __nv_bfloat16* kr = Ks + (wbase + r * 4 + gi) * D;
+        float kf[DPL];
+#pragma unroll
+        for (int part = 0; part < DPL / 8; ++part) {
+          const uint4 v = *reinterpret_cast<const uint4*>(kr + part * 64 + li * 8);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            kf[part * 8 + 2 * e] = bf16lo(w[e]);
+            kf[part * 8 + 2 * e + 1] = bf16hi(w[e]);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float dot = 0.f;
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) dot = fmaf(qf[h][e], kf[e], dot);
+          dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+          dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+          dot += __shfl_xor_sync(0xffffffffu, dot, 4);
+          sc[r][h] = (r * 4 + gi < nw) ? dot : -INFINITY;
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float mx = sc[0][h];
+#pragma unroll
+        for (int r = 1; r < kRounds; ++r) mx = fmaxf(mx, sc[r][h]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float mnew = fmaxf(m[h], mx);
+        const float alpha = fast_exp2(m[h] - mnew);
+        m[h] = mnew;
+        float psum = 0.f;
+#pragma unroll
+        for (int r = 0; r < kRounds; ++r) {
+          const float pr = fast_exp2(sc[r][h] - mnew);
+          sc[r][h] = pr;
+          psum += pr;
+        }
+        l[h] = l[h] * alpha + psum;
+#pragma unroll
+        for (int c = 0; c < DPV; ++c) acc[h][c] *= alpha;
+      }
+      if (li == 0) {
+#pragma unroll
+        for (int r = 0; r < kRounds; ++r)
+#pragma unroll
+          for (int h = 0; h < G; ++h) pw[(r * 4 + gi) * G + h] = sc[r][h];
+      }
+      __syncwarp();
+      const __nv_bfloat16* Vs = sV + (static_cast<size_t>(s) * kTile + wbase) * D + lane * DPV;
+#pragma unroll 4
+      for (int t = 0; t < nw; ++t) {
+        float pv[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) pv[h] = pw[t * G + h];
+        float vf[DPV];
+        if constexpr (DPV == 4) {
+          const uint2 v = *reinterpret_cast<const uint2*>(Vs + t * D);
+          vf[0] = bf16lo(v.x); vf[1] = bf16hi(v.x); vf[2] = bf16lo(v.y); vf[3] = bf16hi(v.y);
+        } else {
+          const uint32_t v = *reinterpret_cast<const uint32_t*>(Vs + t * D);
+          vf[0] = bf16lo(v); vf[1] = bf16hi(v);
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int c = 0; c < DPV; ++c) acc[h][c] = fmaf(pv[h], vf[c], acc[h][c]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+
+  // ---------------------------------------------------- merge the four warps --
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 8);
+    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 16);
+  }
+  float* mw = mrg + warp * G * (D + 2);
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int c = 0; c < DPV; ++c) mw[h * D + lane * DPV + c] = acc[h][c];
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      mw[G * D + 2 * h] = m[h];
+      mw[G * D + 2 * h + 1] = l[h];
+    }
+  }
+  named_barrier_sync(1, kWarps * 32);
+  for (int i = threadIdx.x; i < G * D; i += kWarps * 32) {
+    const int h = i / D, d = i % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mrg[w * G * (D + 2) + G * D + 2 * h]);
+    float lsum = 0.f, o = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float* mwv = mrg + w * G * (D + 2);
+      const float f = fast_exp2(mwv[G * D + 2 * h] - M);
+      lsum += mwv[G * D + 2 * h + 1] * f;
+      o += mwv[h * D + d] * f;
+    }
+    const int64_t row = static_cast<int64_t>(b) * p.num_heads + hq0 + h;
+    if (nchunks == 1) {
+      p.out[row * D + d] = __float2bfloat16(o / lsum);
+    } else {
+      const int64_t idx = row * p.max_chunks + chunk;
+      p.ws_acc[idx * D + d] = o;
+      if (d == 0) {
+        p.ws_ml[2 * idx] = M;
+        p.ws_ml[2 * idx + 1] = lsum;
+      }
+    }
+  }
+}
+
+// Merge of split-KV partials: one warp per (sequence, query head).
+//   M = max_c m_c,  out = sum_c 2^(m_c - M) acc_c / sum_c 2^(m_c - M) l_c
+template <int D>
+__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p, int32_t num_rows) {
+  constexpr int DPV = D / 32;
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= num_rows) return;
+  const int b = row / p.num_heads;
+  const int L = clamp_context(__ldg(p.context_lens + b), p);
+  const int n = (L + p.chunk_tokens - 1) / p.chunk_tokens;
+  if (n <= 1) return;   // written directly by the split kernel (or zero)
+  const float* ml = p.ws_ml + static_cast<int64_t>(row) * p.max_chunks * 2;
+  const float* acc = p.ws_acc + static_cast<int64_t>(row) * p.max_chunks * D;
+  float M = -INFINITY;
+  for (int c = lane; c < n; c += 32) M = fmaxf(M, ml[2 * c]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float lsum = 0.f, o[DPV];
+#pragma unroll
+  for (int c = 0; c < DPV; ++c) o[c] = 0.f;
+  for (int c = 0; c < n; ++c) {
+    const float f = fast_exp2(ml[2 * c] - M);
+    lsum += ml[2 * c + 1] * f;
+    if constexpr (DPV == 4) {
+      const float4 a = *reinterpret_cast<const float4*>(acc + static_cast<int64_t>(c) * D + lane * 4);
+      o[0] += a.x * f; o[1] += a.y * f; o[2] += a.z * f; o[3] += a.w * f;
+    } else {
+      const float2 a = *reinterpret_cast<const float2*>(acc + static_cast<int64_t>(c) * D + lane * 2);
+      o[0] += a.x * f; o[1] += a.y * f;
+    }
+  }
+  const float inv = 1.f / lsum;
+  __nv_bfloat16* out = p.out + static_cast<int64_t>(row) * D + lane * DPV;
+#pragma unroll
+  for (int c = 0; c < DPV; c += 2)
+    *reinterpret_cast<uint32_t*>(out + c) = pack_bf16x2(o[c] * inv, o[c + 1] * inv);
+}
+
+template <int D, int G>
+pa_status launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, dim3 grid,
+                       cudaStream_t stream) {
+  using Smem = DecodeSmem<D, G>;
+  static int configured_device = -1;
+  const DeviceInfo* di = current_device_info();
+  if (configured_device != di->device) {
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(Smem::bytes));
+    if (e != cudaSuccess) {
+      set_last_error("cudaFuncSetAttribute(decode): %s", cudaGetErrorString(e));
+      return PA_ERR_CUDA;
+    }
+    configured_device = di->device;
+  }
+  decode_split_kernel<D, G><<<grid, kThreads, Smem::bytes, stream>>>(tmK, tmV, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error("decode launch: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+template <int D>
+pa_status dispatch_group(int G, const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, dim3 grid,
+                         cudaStream_t stream) {
+  switch (G) {
+    case 1: return launch_split<D, 1>(tmK, tmV, p, grid, stream);
+    case 2: return launch_split<D, 2>(tmK, tmV, p, grid, stream);
+    case 3: return launch_split<D, 3>(tmK, tmV, p, grid, stream);
+    case 4: return launch_split<D, 4>(tmK, tmV, p, grid, stream);
+    case 5: return launch_split<D, 5>(tmK, tmV, p, grid, stream);
+    case 6: return launch_split<D, 6>(tmK, tmV, p, grid, stream);
+    case 7: return launch_split<D, 7>(tmK, tmV, p, grid, stream);
+    case 8: return launch_split<D, 8>(tmK, tmV, p, grid, stream);
+    default: break;
+  }
+  set_last_error("decode: query heads per kv head = %d is not supported (1..8)", G);
+  return PA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+int32_t decode_auto_chunk(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int sm_count) {
+  // Enough CTAs to fill every SM several times over, without chunks so short
+  // that per-CTA set-up dominates.
+  constexpr int kMinChunk = 512;
+  constexpr int kWavesTarget = 4;
+  const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
+  if (max_context_len <= kMinChunk || units <= 0) return ((max(max_context_len, 1) + kTile - 1) / kTile) * kTile;
+  const int64_t want = static_cast<int64_t>(kWavesTarget) * sm_count;
+  int64_t splits = (want + units - 1) / units;
+  const int64_t max_splits = (max_context_len + kMinChunk - 1) / kMinChunk;
+  splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);
+  const int64_t per = (max_context_len + splits - 1) / splits;
+  return static_cast<int32_t>(((per + kTile - 1) / kTile) * kTile);
+}
+
+pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  const int G = a.num_heads / a.num_kv_heads;
+  const int box_rows = a.block_size < kTile ? a.block_size : kTile;
+  CUtensorMap tmK, tmV;
+  const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.block_size;
+  const uint64_t s1 = static_cast<uint64_t>(a.head_dim) * 2;
+  const uint64_t s2 = s1 * a.num_kv_heads;
+  if (!encode_bf16_3d(&tmK, a.k_cache, a.head_dim, a.num_kv_heads, rows, s1, s2, a.head_dim, 1, box_rows,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_bf16_3d(&tmV, a.v_cache, a.head_dim, a.num_kv_heads, rows, s1, s2, a.head_dim, 1, box_rows,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    return PA_ERR_INVALID_ARG;
+  DecodeParams p;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.block_tables = a.block_tables;
+  p.context_lens = a.context_lens;
+  p.ws_acc = a.ws_acc;
+  p.ws_ml = a.ws_ml;
+  p.max_blocks_per_seq = a.max_blocks_per_seq;
+  p.max_context_len = a.max_context_len;
+  p.num_heads = a.num_heads;
+  p.block_size = a.block_size;
+  p.box_rows = box_rows;
+  p.chunk_tokens = a.chunk_tokens;
+  p.max_chunks = a.max_chunks;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.err = current_device_info()->error_word;
+  const dim3 grid(static_cast<unsigned>(a.max_chunks), static_cast<unsigned>(a.num_kv_heads),
+                  static_cast<unsigned>(a.num_seqs));
+  pa_status st = a.head_dim == 128 ? dispatch_group<128>(G, tmK, tmV, p, grid, stream)
+                                   : dispatch_group<64>(G, tmK, tmV, p, grid, stream);
+  if (st != PA_OK || a.max_chunks <= 1) return st;
+  const int32_t rows_out = a.num_seqs * a.num_heads;
+  const unsigned mblocks = static_cast<unsigned>((rows_out + 3) / 4);
+  if (a.head_dim == 128)
+    decode_merge_kernel<128><<<mblocks, 128, 0, stream>>>(p, rows_out);
+  else
+    decode_merge_kernel<64><<<mblocks, 128, 0, stream>>>(p, rows_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error("decode merge launch: %s", cudaGetErrorString(e));
+    return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+}  // namespace pa

@@ -1,0 +1,305 @@
+// C ABI of the paged-KV attention library: argument validation, tensor-map
+// encoding and dispatch to the kernels.  Nothing here allocates device
+// memory; every buffer belongs to the caller.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+// One error word per device that loads the library; kernels record a code
+// here instead of hanging when a pipeline wait runs out of time.
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+thread_local char t_last_error[512] = "";
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_devinfo[kMaxDevices];
+std::once_flag g_devinfo_once[kMaxDevices];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool is_pow2(int32_t x) { return x > 0 && (x & (x - 1)) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pa_status fail(pa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof t_last_error, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+// Shape rules shared by decode and prefill.
+pa_status check_cache_shape(const char* who, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                            int32_t block_size, int32_t num_blocks) {
+  if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads)
+    return fail(PA_ERR_INVALID_ARG, "%s: num_heads (%d) must be a positive multiple of num_kv_heads (%d)", who,
+                num_heads, num_kv_heads);
+  if (num_blocks <= 0) return fail(PA_ERR_INVALID_ARG, "%s: num_blocks must be positive", who);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "%s: head_dim %d not supported (64 or 128)", who, head_dim);
+  if (!is_pow2(block_size) || block_size < 16 || block_size > 1024)
+    return fail(PA_ERR_UNSUPPORTED, "%s: block_size %d not supported (power of two in [16, 1024])", who,
+                block_size);
+  if (static_cast<int64_t>(num_blocks) * block_size >= (int64_t(1) << 31))
+    return fail(PA_ERR_UNSUPPORTED, "%s: num_blocks * block_size must stay below 2^31", who);
+  return PA_OK;
+}
+
+}  // namespace
+
+void set_last_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof t_last_error, fmt, ap);
+  va_end(ap);
+}
+
+const DeviceInfo* current_device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  std::call_once(g_devinfo_once[dev], [dev] {
+    DeviceInfo& d = g_devinfo[dev];
+    d.device = dev;
+    d.sm_count = 148;
+    d.max_smem_optin = 227 * 1024;
+    cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    d.error_word = nullptr;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_device_error) == cudaSuccess) d.error_word = static_cast<unsigned int*>(addr);
+  });
+  return &g_devinfo[dev];
+}
+
+bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                    uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2,
+                    CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) {
+    set_last_error("cuTensorMapEncodeTiled is not available from the driver");
+    return false;
+  }
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_last_error("cuTensorMapEncodeTiled failed (%d): dims %llu x %llu x %llu, box %u x %u x %u", (int)r,
+                   (unsigned long long)d0, (unsigned long long)d1, (unsigned long long)d2, b0, b1, b2);
+    return false;
+  }
+  return true;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char* pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+    default: return "PA_ERR_UNKNOWN";
+  }
+}
+
+const char* pa_last_error(void) { return t_last_error; }
+
+int32_t pa_version(void) { return (1 << 16) | 0; }
+
+pa_status pa_store_kvcache(const void* key, const void* value, int64_t key_row_stride, int64_t value_row_stride,
+                           void* k_cache, void* v_cache, const int32_t* slot_mapping, int32_t num_tokens,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                           void* stream) {
+  t_last_error[0] = 0;
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "store_kvcache: num_tokens < 0");
+  if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "store_kvcache: num_kv_heads, head_dim, block_size, num_blocks must be > 0");
+  const int64_t row = static_cast<int64_t>(num_kv_heads) * head_dim;
+  if (row > (int64_t(1) << 20)) return fail(PA_ERR_UNSUPPORTED, "store_kvcache: row of %lld elements too long",
+                                            (long long)row);
+  if (key_row_stride < row || value_row_stride < row)
+    return fail(PA_ERR_INVALID_ARG, "store_kvcache: row strides must be >= num_kv_heads*head_dim");
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping)
+    return fail(PA_ERR_INVALID_ARG, "store_kvcache: null pointer");
+  const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  cudaError_t e = launch_store_kvcache(key, value, key_row_stride, value_row_stride, k_cache, v_cache, slot_mapping,
+                                       num_tokens, static_cast<int32_t>(row), num_slots,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "store_kvcache launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
+int32_t pa_decode_chunk_size(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int32_t block_size) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || max_context_len < 0 || block_size <= 0) return -1;
+  return decode_auto_chunk(num_seqs, num_kv_heads, max_context_len, current_device_info()->sm_count);
+}
+
+static int32_t resolve_chunk(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int32_t kv_chunk_size) {
+  if (kv_chunk_size == 0)
+    return decode_auto_chunk(num_seqs, num_kv_heads, max_context_len, current_device_info()->sm_count);
+  return kv_chunk_size;
+}
+
+static int32_t chunks_for(int32_t max_context_len, int32_t chunk) {
+  if (max_context_len <= 0) return 1;
+  const int64_t n = (static_cast<int64_t>(max_context_len) + chunk - 1) / chunk;
+  return static_cast<int32_t>(n < 1 ? 1 : n);
+}
+
+static size_t workspace_bytes_for(int32_t num_seqs, int32_t num_heads, int32_t head_dim, int32_t nchunks) {
+  if (nchunks <= 1) return 0;
+  const size_t rows = static_cast<size_t>(num_seqs) * num_heads * nchunks;
+  const size_t acc = (rows * head_dim * sizeof(float) + 255) / 256 * 256;
+  return acc + rows * 2 * sizeof(float);
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t block_size, int32_t kv_chunk_size) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+      block_size <= 0 || kv_chunk_size < 0 || (kv_chunk_size % kDecodeTile))
+    return 0;
+  const int32_t chunk = resolve_chunk(num_seqs, num_kv_heads, max_context_len, kv_chunk_size);
+  return workspace_bytes_for(num_seqs, num_heads, head_dim, chunks_for(max_context_len, chunk));
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                    int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t kv_chunk_size,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  t_last_error[0] = 0;
+  if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "decode: num_seqs < 0");
+  pa_status st = check_cache_shape("decode", num_heads, num_kv_heads, head_dim, block_size, num_blocks);
+  if (st != PA_OK) return st;
+  if (max_context_len < 0 || max_blocks_per_seq <= 0)
+    return fail(PA_ERR_INVALID_ARG, "decode: max_context_len must be >= 0 and max_blocks_per_seq > 0");
+  if (kv_chunk_size < 0 || kv_chunk_size % kDecodeTile)
+    return fail(PA_ERR_INVALID_ARG, "decode: kv_chunk_size must be 0 or a positive multiple of %d", kDecodeTile);
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "decode: scale must be finite and > 0");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PA_ERR_INVALID_ARG, "decode: null pointer");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG, "decode: q, out, k_cache and v_cache must be 16-byte aligned");
+  if (static_cast<int64_t>(num_seqs) > 65535) return fail(PA_ERR_UNSUPPORTED, "decode: more than 65535 sequences");
+  const int32_t chunk = resolve_chunk(num_seqs, num_kv_heads, max_context_len, kv_chunk_size);
+  const int32_t nchunks = chunks_for(max_context_len, chunk);
+  const size_t need = workspace_bytes_for(num_seqs, num_heads, head_dim, nchunks);
+  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(PA_ERR_WORKSPACE, "decode: workspace of %zu bytes (16-byte aligned) required, got %zu", need,
+                workspace ? workspace_bytes : (size_t)0);
+  DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  const size_t rows = static_cast<size_t>(num_seqs) * num_heads * nchunks;
+  a.ws_acc = static_cast<float*>(workspace);
+  a.ws_ml = need ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                            (rows * head_dim * sizeof(float) + 255) / 256 * 256)
+                 : nullptr;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.max_context_len = max_context_len;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.chunk_tokens = chunk;
+  a.max_chunks = nchunks;
+  a.scale = scale;
+  return launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_prefill_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t total_q,
+                            int32_t max_seqlen_q, int32_t max_seqlen_k, const int32_t* block_tables,
+                            int32_t max_blocks_per_seq, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                            int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t causal,
+                            void* stream) {
+  t_last_error[0] = 0;
+  if (num_seqs < 0 || total_q < 0) return fail(PA_ERR_INVALID_ARG, "prefill: num_seqs and total_q must be >= 0");
+  pa_status st = check_cache_shape("prefill", num_heads, num_kv_heads, head_dim, block_size, num_blocks);
+  if (st != PA_OK) return st;
+  const int G = num_heads / num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(PA_ERR_UNSUPPORTED, "prefill: query heads per kv head = %d not supported (1, 2, 4, 8)", G);
+  if (max_seqlen_q < 0 || max_seqlen_k < max_seqlen_q || max_blocks_per_seq <= 0)
+    return fail(PA_ERR_INVALID_ARG, "prefill: need 0 <= max_seqlen_q <= max_seqlen_k and max_blocks_per_seq > 0");
+  if (!(scale > 0.f) || !isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "prefill: scale must be finite and > 0");
+  if (num_seqs == 0 || total_q == 0 || max_seqlen_q == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !cu_seqlens_q || !cu_seqlens_k || !block_tables)
+    return fail(PA_ERR_INVALID_ARG, "prefill: null pointer");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG, "prefill: q, out, k_cache and v_cache must be 16-byte aligned");
+  if (num_seqs > 65535) return fail(PA_ERR_UNSUPPORTED, "prefill: more than 65535 sequences");
+  PrefillArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.cu_seqlens_q = cu_seqlens_q;
+  a.cu_seqlens_k = cu_seqlens_k;
+  a.block_tables = block_tables;
+  a.total_q = total_q;
+  a.max_seqlen_q = max_seqlen_q;
+  a.max_seqlen_k = max_seqlen_k;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.scale = scale;
+  a.causal = causal;
+  return launch_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_device_error(int32_t* code_out, void* stream) {
+  t_last_error[0] = 0;
+  if (!code_out) return fail(PA_ERR_INVALID_ARG, "device_error: null code_out");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof v, 0, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "device_error: %s", cudaGetErrorString(e));
+  *code_out = static_cast<int32_t>(v);
+  return PA_OK;
+}
+
+}  // extern "C"

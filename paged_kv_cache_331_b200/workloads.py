@@ -23,6 +23,7 @@ new K/V rows.
 from __future__ import annotations
 
 import math
+import os
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -45,13 +46,31 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
-def randn_bf16(rng: np.random.Generator, shape, chunk: int = 1 << 24) -> np.ndarray:
-    """N(0,1) draws rounded to bf16, generated in chunks to bound host memory."""
+def randn_bf16(rng: np.random.Generator, shape, chunk: int = 1 << 22) -> np.ndarray:
+    """N(0,1) draws rounded to bf16.
+
+    One 63-bit seed is drawn from ``rng``; chunk i of the flattened tensor is
+    then drawn from ``default_rng([seed, i])``.  The chunks are independent, so
+    they are generated on several host threads; the result depends only on
+    ``rng``'s state and the shape.
+    """
     n = int(np.prod(shape))
+    seed = int(rng.integers(0, 2**63 - 1))
     out = np.empty(n, dtype=np.uint16)
-    for s in range(0, n, chunk):
+    starts = list(range(0, n, chunk))
+
+    def fill(i):
+        s = starts[i]
         e = min(n, s + chunk)
-        out[s:e] = f32_to_bf16_bits(rng.standard_normal(e - s, dtype=np.float32))
+        out[s:e] = f32_to_bf16_bits(np.random.default_rng([seed, i]).standard_normal(e - s, dtype=np.float32))
+
+    if len(starts) <= 2:
+        for i in range(len(starts)):
+            fill(i)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 4, 32)) as ex:
+            list(ex.map(fill, range(len(starts))))
     return out.reshape(shape)
 
 

@@ -1,0 +1,86 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function
+that include/pa.h declares, and rejects bad arguments on the host before any
+launch (no compute calls here)."""
+import ctypes
+import re
+import subprocess
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parent.parent
+HEADER = ROOT / "include" / "pa.h"
+
+
+@pytest.fixture(scope="module")
+def libpa():
+    from paged_kv_cache_331_b200 import build as B
+    B.build()
+    from paged_kv_cache_331_b200 import _binding
+    return _binding.lib()
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("pa_store_kvcache", "pa_decode", "pa_decode_workspace_size", "pa_prefill_varlen"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(libpa):
+    so = ROOT / "paged_kv_cache_331_b200" / "libpagedattn.so"
+    out = subprocess.run(["nm", "-D", "--defined-only", str(so)], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(libpa, n)
+    # nothing else of ours leaks out of the library
+    ours = sorted(n for n in exported if n.startswith("pa_") or "pa::" in n)
+    assert set(ours) <= set(declared_functions())
+
+
+def test_status_strings(libpa):
+    assert libpa.pa_status_string(0) == b"PA_OK"
+    assert libpa.pa_status_string(1) == b"PA_ERR_INVALID_ARG"
+    assert libpa.pa_status_string(4) == b"PA_ERR_WORKSPACE"
+    assert libpa.pa_version() >> 16 == 1
+
+
+def test_host_side_argument_checks(libpa):
+    L = libpa
+    null = None
+    # store: negative token count, short row stride
+    assert L.pa_store_kvcache(null, null, 64, 64, null, null, null, -1, 1, 64, 16, 4, null) == 1
+    assert L.pa_store_kvcache(null, null, 10, 64, null, null, null, 1, 1, 64, 16, 4, null) == 1
+    assert L.pa_store_kvcache(null, null, 64, 64, null, null, null, 0, 1, 64, 16, 4, null) == 0   # nothing to do
+    # decode: group size, head_dim, block size, chunk size
+    args = lambda hq, hkv, d, bs, chunk: (null, null, null, null, null, 4, null, 100, 2, hq, hkv, d, bs, 8, 0.125,
+                                          chunk, null, 0, null)
+    assert L.pa_decode(*args(6, 4, 64, 16, 0)) == 1          # 6 % 4 != 0
+    assert L.pa_decode(*args(4, 2, 96, 16, 0)) == 2          # head_dim 96 unsupported
+    assert L.pa_decode(*args(4, 2, 64, 48, 0)) == 2          # block_size not a power of two
+    assert L.pa_decode(*args(4, 2, 64, 16, 100)) == 1        # chunk not a multiple of 64
+    assert L.pa_decode(*args(4, 2, 64, 16, 64)) == 1         # null pointers
+    assert b"null" in L.pa_last_error()
+    # prefill: unsupported group size, inconsistent max lengths
+    pargs = lambda hq, hkv, mq, mk: (null, null, null, null, null, null, 10, mq, mk, null, 4, 2, hq, hkv, 64, 16, 8,
+                                     0.125, 1, null)
+    assert L.pa_prefill_varlen(*pargs(6, 2, 8, 8)) == 2      # G = 3
+    assert L.pa_prefill_varlen(*pargs(4, 2, 9, 8)) == 1      # max_seqlen_q > max_seqlen_k
+
+
+def test_workspace_size_arithmetic(libpa):
+    """Explicit chunk size: partial (acc, m, l) rows for every (seq, head, chunk)."""
+    B, H, Hkv, D = 3, 8, 2, 128
+    n = libpa.pa_decode_workspace_size(B, H, Hkv, D, 1000, 16, 256)
+    chunks = 4
+    rows = B * H * chunks
+    assert n == (rows * D * 4 + 255) // 256 * 256 + rows * 2 * 4
+    assert libpa.pa_decode_workspace_size(B, H, Hkv, D, 256, 16, 256) == 0     # one chunk: no workspace
+    assert libpa.pa_decode_workspace_size(B, H, Hkv, D, 1000, 16, 100) == 0    # invalid chunk -> 0

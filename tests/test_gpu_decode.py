@@ -1,0 +1,108 @@
+"""Paged GQA decode (and its split-KV merge) on the GPU against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_331_b200 as pa
+from paged_kv_cache_331_b200 import workloads as W
+from gpu_helpers import DeviceDecode, assert_attention_close, host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def store_and_decode(dw, kv_chunk_size=0):
+    w = dw.w
+    pa.store_kvcache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping)
+    out = pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.context_lens, w.max_context_len, w.scale,
+                    kv_chunk_size=kv_chunk_size)
+    torch.cuda.synchronize()
+    return out
+
+
+def oracle_decode(oracle, w):
+    oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
+    _, of = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
+    return of
+
+
+CASES = [
+    # lens, hq, hkv, d, bs
+    ([1, 17, 256, 300], 4, 2, 64, 256),
+    ([5, 33, 64, 1, 100, 0, 129], 8, 2, 128, 16),
+    ([200, 64, 65, 63], 3, 1, 128, 32),
+    ([700, 1], 5, 1, 64, 64),
+    ([333, 1000, 2], 8, 1, 128, 128),
+    ([1500, 257], 16, 2, 128, 1024),
+    ([90, 91, 92], 6, 1, 64, 16),
+    ([130, 7], 7, 1, 128, 256),
+    ([640, 100], 2, 2, 64, 512),
+]
+
+
+@pytest.mark.parametrize("lens,hq,hkv,d,bs", CASES)
+@pytest.mark.parametrize("chunk", [0, 64, 192, 512])
+def test_decode_small_shapes(oracle, lens, hq, hkv, d, bs, chunk):
+    rng = np.random.default_rng(sum(lens) + hq * 7 + d + bs)
+    w = W.decode_workload(np.array(lens, np.int32), hq, hkv, d, bs, rng=rng)
+    out = store_and_decode(DeviceDecode(w), kv_chunk_size=chunk)
+    ref = oracle_decode(oracle, w)
+    assert_attention_close(out, ref, what=f"decode {lens} G={hq // hkv} D={d} bs={bs} chunk={chunk}")
+    zero_rows = np.asarray(lens) == 0
+    if zero_rows.any():
+        assert not host_bits(out)[zero_rows].any()
+
+
+@pytest.mark.parametrize("make", [W.tiny_decode, W.qwen3_decode, W.large_batch_decode, W.long_context_decode])
+def test_decode_named_workloads_full_size(oracle, make):
+    """Every output element of the full-size workloads, automatic split-KV."""
+    w = make()
+    dw = DeviceDecode(w)
+    out = store_and_decode(dw)
+    ref = oracle_decode(oracle, w)
+    mx, mean = assert_attention_close(out, ref, what=w.name)
+    print(f"{w.name}: chunk={pa.decode_chunk_size(w.num_seqs, w.num_kv_heads, w.max_context_len, w.block_size)} "
+          f"max_abs={mx:.2e} mean_abs={mean:.2e}")
+
+
+def test_decode_poisoned_cache_and_determinism(oracle):
+    """NaN in every cache row outside the contexts (and in unused blocks) changes nothing; repeat runs are
+    bitwise identical."""
+    rng = np.random.default_rng(31)
+    lens = np.array([700, 3, 129, 64, 1, 250], np.int32)
+    w = W.decode_workload(lens, 8, 2, 128, 64, rng=rng, poison_unused=True)
+    # the new rows are stored into poisoned slots first
+    dw = DeviceDecode(w)
+    out1 = store_and_decode(dw, kv_chunk_size=128)
+    out2 = pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.context_lens, w.max_context_len, w.scale,
+                     kv_chunk_size=128)
+    torch.cuda.synchronize()
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    ref = oracle_decode(oracle, w)
+    assert_attention_close(out1, ref, what="poisoned")
+
+
+def test_decode_block_table_padding_never_read(oracle):
+    """Entries past ceil(L / block_size) hold -1 (and the table is wider than needed)."""
+    rng = np.random.default_rng(32)
+    w = W.decode_workload(np.array([40, 17], np.int32), 4, 2, 64, 16, rng=rng)
+    wide = np.full((2, 64), -1, np.int32)
+    wide[:, :w.block_tables.shape[1]] = w.block_tables
+    w.block_tables = wide
+    out = store_and_decode(DeviceDecode(w))
+    assert_attention_close(out, oracle_decode(oracle, w), what="padded table")
+
+
+def test_decode_workspace_too_small_is_rejected():
+    rng = np.random.default_rng(33)
+    w = W.decode_workload(np.array([1000], np.int32), 4, 2, 64, 16, rng=rng)
+    dw = DeviceDecode(w)
+    need = pa.decode_workspace_size(1, 4, 2, 64, 1000, 16, 64)
+    assert need > 0
+    small = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pa.PagedAttentionError, match="WORKSPACE"):
+        pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.context_lens, 1000, w.scale,
+                  kv_chunk_size=64, workspace=small)
+
+
+def test_decode_no_device_error():
+    assert pa.device_error() == 0

@@ -1,0 +1,92 @@
+"""Varlen causal prefill with prefix-cache blocks on the GPU against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_331_b200 as pa
+from paged_kv_cache_331_b200 import workloads as W
+from gpu_helpers import DevicePrefill, assert_attention_close, host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def store_and_prefill(dp):
+    w = dp.w
+    pa.store_kvcache(dp.new_k, dp.new_v, dp.k_cache, dp.v_cache, dp.slot_mapping)
+    out = pa.prefill_varlen(dp.q, dp.k_cache, dp.v_cache, dp.cu_seqlens_q, dp.cu_seqlens_k, w.max_seqlen_q,
+                            w.max_seqlen_k, dp.block_tables, w.scale, w.causal)
+    torch.cuda.synchronize()
+    return out
+
+
+def oracle_prefill(oracle, w, row_select=None):
+    oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
+    _, of = oracle.prefill_varlen(w.q, w.k_cache, w.v_cache, w.cu_seqlens_q, w.cu_seqlens_k, w.block_tables, w.scale,
+                                  w.causal, row_select=row_select, want_f64=True)
+    return of
+
+
+CASES = [
+    # prefix, suffixes, hq, hkv, d, bs, causal
+    (0, [5, 17, 1], 4, 2, 64, 16, True),
+    (0, [128, 129, 300], 2, 1, 128, 256, True),
+    (256, [64, 1, 200], 16, 8, 128, 256, True),
+    (32, [9, 20, 150], 4, 1, 128, 16, True),
+    (64, [40, 3, 130], 8, 1, 64, 32, True),
+    (128, [77, 255], 8, 8, 128, 128, True),
+    (512, [300, 64], 16, 2, 128, 64, True),
+    (32, [9, 20], 4, 4, 64, 16, False),
+    (256, [100, 257], 8, 2, 128, 256, False),
+]
+
+
+@pytest.mark.parametrize("prefix,sfx,hq,hkv,d,bs,causal", CASES)
+def test_prefill_small_shapes(oracle, prefix, sfx, hq, hkv, d, bs, causal):
+    rng = np.random.default_rng(prefix + sum(sfx) + hq + d + bs)
+    w = W.prefill_workload(prefix, np.array(sfx, np.int32), hq, hkv, d, bs, rng=rng, causal=causal)
+    out = store_and_prefill(DevicePrefill(w))
+    ref = oracle_prefill(oracle, w)
+    assert_attention_close(out, ref, what=f"prefill prefix={prefix} sfx={sfx} G={hq // hkv} D={d} bs={bs}")
+
+
+def test_prefill_prefix_workload_full_size_sampled(oracle):
+    """The 32-sequence prefix-cached workload at full size; the oracle checks every 5th query token plus the
+    first and last token of every sequence (all heads)."""
+    w = W.prefix_prefill()
+    out = store_and_prefill(DevicePrefill(w))
+    T = int(w.cu_seqlens_q[-1])
+    sel = np.zeros(T, np.uint8)
+    sel[::5] = 1
+    sel[w.cu_seqlens_q[:-1]] = 1
+    sel[w.cu_seqlens_q[1:] - 1] = 1
+    ref = oracle_prefill(oracle, w, row_select=sel)
+    mx, mean = assert_attention_close(out, ref, mask=sel.astype(bool), what="prefix_prefill (sampled)")
+    print(f"prefix prefill: {int(sel.sum())} of {T} tokens checked, max_abs={mx:.2e} mean_abs={mean:.2e}")
+
+
+def test_prefill_shared_vs_duplicated_prefix_identical():
+    """Prefix blocks shared by every block table give bitwise the same output as private copies."""
+    a = W.prefill_workload(512, np.array([100, 37, 300], np.int32), 16, 8, 128, 256,
+                           rng=np.random.default_rng(41), shared_prefix=True)
+    b = W.prefill_workload(512, np.array([100, 37, 300], np.int32), 16, 8, 128, 256,
+                           rng=np.random.default_rng(41), shared_prefix=False)
+    for s in range(3):
+        Lk = int(a.cu_seqlens_k[s + 1] - a.cu_seqlens_k[s])
+        for p in range(0, Lk, 256):
+            b.k_cache[b.block_tables[s, p // 256]] = a.k_cache[a.block_tables[s, p // 256]]
+            b.v_cache[b.block_tables[s, p // 256]] = a.v_cache[a.block_tables[s, p // 256]]
+    b.q[:] = a.q; b.new_k[:] = a.new_k; b.new_v[:] = a.new_v
+    oa = store_and_prefill(DevicePrefill(a))
+    ob = store_and_prefill(DevicePrefill(b))
+    assert torch.equal(oa.view(torch.int16), ob.view(torch.int16))
+
+
+def test_prefill_poisoned_cache(oracle):
+    rng = np.random.default_rng(42)
+    w = W.prefill_workload(64, np.array([50, 130, 7], np.int32), 8, 2, 128, 64, rng=rng, poison_unused=True)
+    out = store_and_prefill(DevicePrefill(w))
+    assert_attention_close(out, oracle_prefill(oracle, w), what="poisoned prefill")
+
+
+def test_prefill_no_device_error():
+    assert pa.device_error() == 0
