@@ -38,7 +38,6 @@ constexpr int kTile = kDecodeTile;         // tokens per stage
 constexpr int kWarps = 4;                  // consumer warps
 constexpr int kTPW = kTile / kWarps;       // tokens per consumer warp per tile
 constexpr int kRounds = kTPW / 4;          // QK rounds (4 tokens per warp per round)
-constexpr int kStages = 4;
 constexpr int kThreads = (kWarps + 1) * 32;
 
 struct DecodeParams {
@@ -59,16 +58,24 @@ struct DecodeParams {
   unsigned int* err;
 };
 
+// Per-shape configuration.  Two CTAs share an SM whenever their shared memory
+// and registers fit, so each SM has eight consumer warps to hide latency.
 template <int D, int G>
-struct DecodeSmem {
+struct DecodeCfg {
+  static constexpr int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));   // group padded to a power of two
+  static constexpr int HB = GP == 1 ? 0 : (GP == 2 ? 1 : (GP == 4 ? 2 : 3)); // log2(GP)
+  static constexpr int kStages = (D == 64) ? 4 : (G <= 4 ? 3 : 4);
+  static constexpr int kMinBlocks = (D == 64 || G <= 4) ? 2 : 1;
   static constexpr size_t kv_stage_elems = static_cast<size_t>(kTile) * D;
   static constexpr size_t k_off = 0;
   static constexpr size_t v_off = k_off + kStages * kv_stage_elems * 2;
   static constexpr size_t p_off = v_off + kStages * kv_stage_elems * 2;
-  static constexpr size_t m_off = p_off + static_cast<size_t>(kWarps) * kTPW * G * 4;
-  static constexpr size_t bar_off = m_off + static_cast<size_t>(kWarps) * G * (D + 2) * 4;
+  static constexpr size_t bar_off = p_off + static_cast<size_t>(kWarps) * kTPW * G * 2 * 4;
   static constexpr size_t bytes = bar_off + 2 * kStages * 8;
-  static_assert(m_off % 8 == 0 && bar_off % 8 == 0, "alignment");
+  // the cross-warp merge area reuses the K stages once every tile is consumed
+  static constexpr size_t merge_bytes = static_cast<size_t>(kWarps) * G * (D + 2) * 4;
+  static_assert(merge_bytes <= kStages * kv_stage_elems * 2, "merge area must fit in the K stages");
+  static_assert(bar_off % 8 == 0, "alignment");
 };
 
 __device__ __forceinline__ int clamp_context(int L, const DecodeParams& p) {
@@ -77,21 +84,67 @@ __device__ __forceinline__ int clamp_context(int L, const DecodeParams& p) {
   return max(L, 0);
 }
 
+// Butterfly reduce-scatter over the 8 lanes of a token group: on entry every
+// lane holds CNT partial dot products (one per head); on exit v[0] holds the
+// full sum for one head, selected by the lane's bits (lane & 4, 2, 1 pick the
+// upper half at each halving step), with CNT-1 fewer shuffles than reducing
+// every head separately.
+template <int CNT, int MASK>
+__device__ __forceinline__ void reduce_scatter(float* v, int lane) {
+  if constexpr (MASK == 0) {
+    return;
+  } else if constexpr (CNT > 1) {
+    constexpr int H = CNT / 2;
+    const bool up = (lane & MASK) != 0;
+#pragma unroll
+    for (int i = 0; i < H; ++i) {
+      const float send = up ? v[i] : v[H + i];
+      const float keep = up ? v[H + i] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, MASK);
+    }
+    reduce_scatter<H, MASK / 2>(v, lane);
+  } else {
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], MASK);
+    reduce_scatter<1, MASK / 2>(v, lane);
+  }
+}
+
+// Head held by lane-in-group li after reduce_scatter<GP, 4>, and the lane that
+// is the canonical holder of head h (its non-head bits zero).
+template <int GP, int HB>
+__device__ __forceinline__ int head_of_lane(int li) {
+  int h = 0;
+#pragma unroll
+  for (int k = 0; k < HB; ++k)
+    if (li & (4 >> k)) h += GP >> (k + 1);
+  return h;
+}
+template <int HB>
+__device__ __forceinline__ int lane_of_head(int h) {
+  int li = 0;
+#pragma unroll
+  for (int k = 0; k < HB; ++k)
+    if ((h >> (HB - 1 - k)) & 1) li |= 4 >> k;
+  return li;
+}
+
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const DecodeParams p) {
-  using Smem = DecodeSmem<D, G>;
+  using Cfg = DecodeCfg<D, G>;
+  constexpr int kStages = Cfg::kStages;
+  constexpr int GP = Cfg::GP, HB = Cfg::HB;
   constexpr int DPL = D / 8;    // query/key dims per lane in QK (8 lanes per token)
   constexpr int DPV = D / 32;   // output dims per lane in PV
   static_assert(D == 64 || D == 128, "head_dim");
 
   extern __shared__ __align__(128) uint8_t smem[];
-  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + Smem::k_off);
-  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + Smem::v_off);
-  float* pbuf = reinterpret_cast<float*>(smem + Smem::p_off);
-  float* mrg = reinterpret_cast<float*>(smem + Smem::m_off);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Smem::bar_off);
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + Cfg::k_off);
+  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + Cfg::v_off);
+  float* pbuf = reinterpret_cast<float*>(smem + Cfg::p_off);
+  float* mrg = reinterpret_cast<float*>(smem + Cfg::k_off);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::bar_off);
   uint64_t* empty = full + kStages;
 
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -156,6 +209,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // -------------------------------------------------------------- consumers --
   const int li = lane & 7, gi = lane >> 3;
+  const int hsel = head_of_lane<GP, HB>(li);            // head whose score this lane ends up with
+  constexpr int kHeadBits = (7 << (3 - HB)) & 7;
+  const bool owner = (li & ~kHeadBits & 7) == 0 && hsel < G;   // one lane per (token, head) writes p
+
+  // q in registers as (even, odd) dim pairs, pre-scaled by scale * log2(e)
   float qf[G][DPL];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -171,15 +229,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  float m[G], l[G], acc[G][DPV];
+  float m[G], acc[G][DPV];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     m[h] = -INFINITY;
-    l[h] = 0.f;
 #pragma unroll
     for (int c = 0; c < DPV; ++c) acc[h][c] = 0.f;
   }
-  float* pw = pbuf + warp * kTPW * G;
+  float m_own = -INFINITY, l_own = 0.f;   // running max / sum of this lane's head (lane-group partial)
+  float* pw = pbuf + warp * kTPW * G * 2;
   const int wbase = warp * kTPW;
 
   for (int it = 0; it < ntiles; ++it) {
@@ -189,66 +247,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nw = min(kTPW, valid - wbase);
     if (nw > 0) {
       const __nv_bfloat16* Ks = sK + static_cast<size_t>(s) * kTile * D;
-      float sc[kRounds][G];
+      float sc[kRounds];
 #pragma unroll
       for (int r = 0; r < kRounds; ++r) {
         const __nv_bfloat16* kr = Ks + (wbase + r * 4 + gi) * D;
-        float kf[DPL];
+        uint32_t kw[DPL / 2];
 #pragma unroll
         for (int part = 0; part < DPL / 8; ++part) {
           const uint4 v = *reinterpret_cast<const uint4*>(kr + part * 64 + li * 8);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          kw[part * 4 + 0] = v.x; kw[part * 4 + 1] = v.y; kw[part * 4 + 2] = v.z; kw[part * 4 + 3] = v.w;
+        }
+        float kf[DPL];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            kf[part * 8 + 2 * e] = bf16lo(w[e]);
-            kf[part * 8 + 2 * e + 1] = bf16hi(w[e]);
+        for (int e = 0; e < DPL / 2; ++e) {
+          kf[2 * e] = bf16lo(kw[e]);
+          kf[2 * e + 1] = bf16hi(kw[e]);
+        }
+        float v[GP];
+#pragma unroll
+        for (int h = 0; h < GP; ++h) {
+          if (h < G) {
+            float e0 = 0.f, e1 = 0.f;
+#pragma unroll
+            for (int e = 0; e < DPL / 2; ++e) ffma2(e0, e1, qf[h][2 * e], qf[h][2 * e + 1], kf[2 * e], kf[2 * e + 1]);
+            v[h] = e0 + e1;
+          } else {
+            v[h] = 0.f;
           }
         }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float dot = 0.f;
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) dot = fmaf(qf[h][e], kf[e], dot);
-          dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-          dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-          dot += __shfl_xor_sync(0xffffffffu, dot, 4);
-          sc[r][h] = (r * 4 + gi < nw) ? dot : -INFINITY;
-        }
+        reduce_scatter<GP, 4>(v, lane);
+        sc[r] = (r * 4 + gi < nw && hsel < G) ? v[0] : -INFINITY;
       }
+      // tile max of every head, visible in every lane
+      float mx = sc[0];
+#pragma unroll
+      for (int r = 1; r < kRounds; ++r) mx = fmaxf(mx, sc[r]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float mx = sc[0][h];
-#pragma unroll
-        for (int r = 1; r < kRounds; ++r) mx = fmaxf(mx, sc[r][h]);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float mnew = fmaxf(m[h], mx);
+        const float mh = __shfl_sync(0xffffffffu, mx, lane_of_head<HB>(h));
+        const float mnew = fmaxf(m[h], mh);
         const float alpha = fast_exp2(m[h] - mnew);
         m[h] = mnew;
-        float psum = 0.f;
 #pragma unroll
-        for (int r = 0; r < kRounds; ++r) {
-          const float pr = fast_exp2(sc[r][h] - mnew);
-          sc[r][h] = pr;
-          psum += pr;
-        }
-        l[h] = l[h] * alpha + psum;
-#pragma unroll
-        for (int c = 0; c < DPV; ++c) acc[h][c] *= alpha;
+        for (int c = 0; c < DPV; c += 2) fmul2(acc[h][c], acc[h][c + 1], alpha, alpha);
       }
-      if (li == 0) {
+      const float m_own_new = fmaxf(m_own, mx);
+      const float a_own = fast_exp2(m_own - m_own_new);
+      m_own = m_own_new;
+      float psum = 0.f;
 #pragma unroll
-        for (int r = 0; r < kRounds; ++r)
-#pragma unroll
-          for (int h = 0; h < G; ++h) pw[(r * 4 + gi) * G + h] = sc[r][h];
+      for (int r = 0; r < kRounds; ++r) {
+        const float pr = fast_exp2(sc[r] - m_own_new);
+        psum += pr;
+        if (owner) *reinterpret_cast<float2*>(pw + ((r * 4 + gi) * G + hsel) * 2) = make_float2(pr, pr);
       }
+      l_own = l_own * a_own + psum;
       __syncwarp();
       const __nv_bfloat16* Vs = sV + (static_cast<size_t>(s) * kTile + wbase) * D + lane * DPV;
 #pragma unroll 4
       for (int t = 0; t < nw; ++t) {
-        float pv[G];
+        float pv[2 * G];
+        if constexpr (G % 2 == 0) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) pv[h] = pw[t * G + h];
+          for (int h = 0; h < G; h += 2) {
+            const float4 x = *reinterpret_cast<const float4*>(pw + (t * G + h) * 2);
+            pv[2 * h] = x.x; pv[2 * h + 1] = x.y; pv[2 * h + 2] = x.z; pv[2 * h + 3] = x.w;
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float2 x = *reinterpret_cast<const float2*>(pw + (t * G + h) * 2);
+            pv[2 * h] = x.x; pv[2 * h + 1] = x.y;
+          }
+        }
         float vf[DPV];
         if constexpr (DPV == 4) {
           const uint2 v = *reinterpret_cast<const uint2*>(Vs + t * D);
@@ -260,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < G; ++h)
 #pragma unroll
-          for (int c = 0; c < DPV; ++c) acc[h][c] = fmaf(pv[h], vf[c], acc[h][c]);
+          for (int c = 0; c < DPV; c += 2) ffma2(acc[h][c], acc[h][c + 1], pv[2 * h], pv[2 * h + 1], vf[c], vf[c + 1]);
       }
     }
     __syncwarp();
@@ -268,11 +341,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---------------------------------------------------- merge the four warps --
+  // every tile has been consumed, so the K stages are free for the merge area
+  l_own += __shfl_xor_sync(0xffffffffu, l_own, 8);
+  l_own += __shfl_xor_sync(0xffffffffu, l_own, 16);
+  float lh[G];
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 8);
-    l[h] += __shfl_xor_sync(0xffffffffu, l[h], 16);
-  }
+  for (int h = 0; h < G; ++h) lh[h] = __shfl_sync(0xffffffffu, l_own, lane_of_head<HB>(h));
+  named_barrier_sync(1, kWarps * 32);   // all warps are past their last read of the K stages
   float* mw = mrg + warp * G * (D + 2);
 #pragma unroll
   for (int h = 0; h < G; ++h)
@@ -282,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       mw[G * D + 2 * h] = m[h];
-      mw[G * D + 2 * h + 1] = l[h];
+      mw[G * D + 2 * h + 1] = lh[h];
     }
   }
   named_barrier_sync(1, kWarps * 32);
@@ -355,19 +430,19 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p,
 template <int D, int G>
 pa_status launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, dim3 grid,
                        cudaStream_t stream) {
-  using Smem = DecodeSmem<D, G>;
+  using Cfg = DecodeCfg<D, G>;
   static int configured_device = -1;
   const DeviceInfo* di = current_device_info();
   if (configured_device != di->device) {
     cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(Smem::bytes));
+                                         static_cast<int>(Cfg::bytes));
     if (e != cudaSuccess) {
       set_last_error("cudaFuncSetAttribute(decode): %s", cudaGetErrorString(e));
       return PA_ERR_CUDA;
     }
     configured_device = di->device;
   }
-  decode_split_kernel<D, G><<<grid, kThreads, Smem::bytes, stream>>>(tmK, tmV, p);
+  decode_split_kernel<D, G><<<grid, kThreads, Cfg::bytes, stream>>>(tmK, tmV, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("decode launch: %s", cudaGetErrorString(e));
@@ -397,13 +472,13 @@ pa_status dispatch_group(int G, const CUtensorMap& tmK, const CUtensorMap& tmV, 
 }  // namespace
 
 int32_t decode_auto_chunk(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int sm_count) {
-  // Enough CTAs to fill every SM several times over, without chunks so short
-  // that per-CTA set-up dominates.
+  // Enough CTAs to fill every CTA slot (two per SM) several times over,
+  // without chunks so short that per-CTA set-up dominates.
   constexpr int kMinChunk = 512;
   constexpr int kWavesTarget = 4;
   const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
   if (max_context_len <= kMinChunk || units <= 0) return ((max(max_context_len, 1) + kTile - 1) / kTile) * kTile;
-  const int64_t want = static_cast<int64_t>(kWavesTarget) * sm_count;
+  const int64_t want = static_cast<int64_t>(kWavesTarget) * 2 * sm_count;
   int64_t splits = (want + units - 1) / units;
   const int64_t max_splits = (max_context_len + kMinChunk - 1) / kMinChunk;
   splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);

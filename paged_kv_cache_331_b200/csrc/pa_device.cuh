@@ -251,6 +251,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Packed fp32 multiply-add on a pair: (d0, d1) = (a0*b0 + d0, a1*b1 + d1),
+// one instruction for two FMAs (fma.rn.f32x2, sm_100).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 A, B, C;\n\t"
+      "mov.b64 A, {%2, %3};\n\t"
+      "mov.b64 B, {%4, %5};\n\t"
+      "mov.b64 C, {%0, %1};\n\t"
+      "fma.rn.f32x2 C, A, B, C;\n\t"
+      "mov.b64 {%0, %1}, C;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Packed fp32 multiply on a pair: (d0, d1) *= (s0, s1).
+__device__ __forceinline__ void fmul2(float& d0, float& d1, float s0, float s1) {
+  asm("{\n\t.reg .b64 A, C;\n\t"
+      "mov.b64 A, {%2, %3};\n\t"
+      "mov.b64 C, {%0, %1};\n\t"
+      "mul.rn.f32x2 C, A, C;\n\t"
+      "mov.b64 {%0, %1}, C;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(s0), "f"(s1));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

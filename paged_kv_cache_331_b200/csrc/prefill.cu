@@ -26,6 +26,10 @@
 // S_{j+1} is issued before waiting for softmax_j, so the tensor core works
 // on the next tile while the softmax runs.
 //
+// The running max moves lazily (only when a row's max grows by more than
+// 2^8), and P is double-buffered, so softmax_{j+1} normally waits for neither
+// PV_j nor an O correction.
+//
 // Every wait is time-limited (pa_device.cuh); on a timeout the kernel records
 // an error code, drains its copies and MMAs, frees TMEM and returns.
 #include <cuda_runtime.h>
@@ -66,10 +70,10 @@ struct PrefillSmem {
   static constexpr size_t q_off = 0;
   static constexpr size_t k_off = q_off + kChunks * kChunkBytes;
   static constexpr size_t v_off = k_off + kStages * kChunks * kChunkBytes;
-  static constexpr size_t p_off = v_off + kStages * kChunks * kChunkBytes;
-  static constexpr size_t bar_off = p_off + 2 * kChunkBytes;
-  // barriers: q_full, kv_full[2], kv_empty[2], s_full[2], p_full, o_done, mma_done
-  static constexpr int kNumBars = 10;
+  static constexpr size_t p_off = v_off + kStages * kChunks * kChunkBytes;   // two P buffers
+  static constexpr size_t bar_off = p_off + 2 * 2 * kChunkBytes;
+  // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_done[2], mma_done
+  static constexpr int kNumBars = 16;
   static constexpr size_t tmem_slot_off = bar_off + kNumBars * 8;
   static constexpr size_t bytes = tmem_slot_off + 16;
   static constexpr size_t alloc_bytes = bytes + 1024;   // slack for 1024-byte alignment
@@ -77,6 +81,28 @@ struct PrefillSmem {
 
 // Byte offset of 16-byte unit u (0..7) of row r inside a 128B-swizzled chunk.
 __device__ __forceinline__ uint32_t sw128(int r, int u) { return r * 128 + ((u ^ (r & 7)) << 4); }
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n\t.reg .b64 A, C;\n\t"
+      "mov.b64 A, {%2, %3};\n\t"
+      "mov.b64 C, {%0, %1};\n\t"
+      "add.rn.f32x2 C, A, C;\n\t"
+      "mov.b64 {%0, %1}, C;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+
+// A row's running max only moves when the tile max exceeds it by more than
+// 2^kRescaleLog2 (in exp2 units); until then the stale max keeps every
+// probability <= 2^kRescaleLog2, exact after the final division, and the O
+// accumulator in TMEM needs no correction.
+constexpr float kRescaleLog2 = 8.0f;
 
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -97,12 +123,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sP = smem + Smem::p_off;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::bar_off);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 3;
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 7;
-  uint64_t* o_done = bars + 8;
-  uint64_t* mma_done = bars + 9;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 3;
+  uint64_t* v_full = bars + 5;
+  uint64_t* v_empty = bars + 7;
+  uint64_t* s_full = bars + 9;
+  uint64_t* p_full = bars + 11;
+  uint64_t* o_done = bars + 13;
+  uint64_t* mma_done = bars + 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::tmem_slot_off);
 
   const int b = blockIdx.z, g = blockIdx.y;
@@ -118,17 +146,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int i_last = min(Lq, (qt + 1) * QP) - 1;
   const int n_keys = p.causal ? min(Lk, pos_off + i_last + 1) : Lk;   // keys any row of the tile may see
   const int nt = (n_keys + kBN - 1) / kBN;
+  // keys every row of the tile sees: tiles entirely below this need no mask
+  const int full_keys = p.causal ? min(Lk, pos_off + qt * QP + 1) : Lk;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], kSoftmaxThreads);
+      mbar_init(&o_done[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, kSoftmaxThreads);
-    mbar_init(o_done, 1);
     mbar_init(mma_done, 1);
     fence_barrier_init();
   }
@@ -154,29 +185,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq;
       const int bs_shift = __ffs(p.block_size) - 1;
       const int nblk_valid = (Lk + p.block_size - 1) >> bs_shift;
-      int issued = 0;
-      for (int j = 0; j < nt; ++j) {
-        const int s = j % kStages;
-        if (!mbar_wait(&kv_empty[s], ((j / kStages) & 1) ^ 1, p.err)) break;
+      // One K or V tile: boxes past the last block of the sequence are skipped
+      // (their table entries may be -1).
+      auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int j) {
         int nbox = kBN / p.box_rows;
-        // skip boxes past the last block of the sequence (their table entries may be -1)
         while (nbox > 0 && ((j * kBN + (nbox - 1) * p.box_rows) >> bs_shift) >= nblk_valid) --nbox;
-        mbar_arrive_expect_tx(&kv_full[s], static_cast<uint32_t>(nbox * p.box_rows * 128 * kChunks * 2));
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox * p.box_rows * 128 * kChunks));
         for (int k = 0; k < nbox; ++k) {
           const int tok = j * kBN + k * p.box_rows;
           const int blk = __ldg(bt + (tok >> bs_shift));
           const int row = (blk << bs_shift) + (tok & (p.block_size - 1));
-          for (int c = 0; c < kChunks; ++c) {
-            const uint32_t off = (s * kChunks + c) * kChunkBytes + k * p.box_rows * 128;
-            tma_load_3d(sK + off, &tmK, &kv_full[s], c * 64, g, row);
-            tma_load_3d(sV + off, &tmV, &kv_full[s], c * 64, g, row);
-          }
+          for (int c = 0; c < kChunks; ++c) tma_load_3d(dst + c * kChunkBytes + k * p.box_rows * 128, map, bar, c * 64, g, row);
         }
-        ++issued;
+      };
+      // K runs one tile ahead of V: K_j's slot frees as soon as S_j is computed,
+      // V_j's only after PV_j.
+      int k_issued = 0, v_issued = 0;
+      bool ok = true;
+      if (nt > 0 && (ok = mbar_wait(&k_empty[0], 1, p.err))) {
+        load_tile(&tmK, sK, &k_full[0], 0);
+        k_issued = 1;
+      }
+      for (int j = 0; ok && j < nt; ++j) {
+        if (j + 1 < nt) {
+          const int s1 = (j + 1) % kStages;
+          if (!(ok = mbar_wait(&k_empty[s1], (((j + 1) / kStages) & 1) ^ 1, p.err))) break;
+          load_tile(&tmK, sK + s1 * kChunks * kChunkBytes, &k_full[s1], j + 1);
+          k_issued = j + 2;
+        }
+        const int s = j % kStages;
+        if (!(ok = mbar_wait(&v_empty[s], ((j / kStages) & 1) ^ 1, p.err))) break;
+        load_tile(&tmV, sV + s * kChunks * kChunkBytes, &v_full[s], j);
+        v_issued = j + 1;
       }
       mbar_wait(q_full, 0, p.err, kErrDrainTimeout);
-      for (int j = max(0, issued - kStages); j < issued; ++j)
-        mbar_wait(&kv_full[j % kStages], (j / kStages) & 1, p.err, kErrDrainTimeout);
+      for (int j = max(0, k_issued - kStages); j < k_issued; ++j)
+        mbar_wait(&k_full[j % kStages], (j / kStages) & 1, p.err, kErrDrainTimeout);
+      for (int j = max(0, v_issued - kStages); j < v_issued; ++j)
+        mbar_wait(&v_full[j % kStages], (j / kStages) & 1, p.err, kErrDrainTimeout);
     }
   } else if (warp == 5) {
     // -------------------------------------------------------------- MMA issuer --
@@ -195,9 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_mma_ss(d_tmem, ad, bd, kIdescS, (c | kk) != 0);
           }
         tc_commit(&s_full[j & 1]);
+        tc_commit(&k_empty[s]);
       };
       if (ok && nt > 0) {
-        ok = mbar_wait(&kv_full[0], 0, p.err);
+        ok = mbar_wait(&k_full[0], 0, p.err);
         if (ok) {
           tc_fence_after();
           issue_s(0);
@@ -206,21 +253,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < nt; ++j) {
         if (j + 1 < nt) {
           const int s1 = (j + 1) % kStages;
-          if (!(ok = mbar_wait(&kv_full[s1], ((j + 1) / kStages) & 1, p.err))) break;
+          if (!(ok = mbar_wait(&k_full[s1], ((j + 1) / kStages) & 1, p.err))) break;
           tc_fence_after();
           issue_s(j + 1);
         }
-        if (!(ok = mbar_wait(p_full, j & 1, p.err))) break;
-        tc_fence_after();
         const int s = j % kStages;
+        if (!(ok = mbar_wait(&v_full[s], (j / kStages) & 1, p.err))) break;
+        if (!(ok = mbar_wait(&p_full[j & 1], (j >> 1) & 1, p.err))) break;
+        tc_fence_after();
+        const uint32_t pb = p_base + (j & 1) * 2 * kChunkBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {   // O += P_j V_j, 16 tokens per MMA
-          const uint64_t ad = smem_desc(p_base + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024, 2);
+          const uint64_t ad = smem_desc(pb + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024, 2);
           const uint64_t bd = smem_desc(v_base + s * kChunks * kChunkBytes + kk * 2048, kChunkBytes, 1024, 2);
           tc_mma_ss(tmem + kColO, ad, bd, kIdescO, (j | kk) != 0);
         }
-        tc_commit(o_done);
-        tc_commit(&kv_empty[s]);
+        tc_commit(&o_done[j & 1]);
+        tc_commit(&v_empty[s]);
       }
       // wait for every MMA this thread issued before TMEM can be released
       tc_commit(mma_done);
@@ -234,47 +283,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_valid = i < Lq;
     const int p_row = p.causal ? min(pos_off + i, Lk - 1) : Lk - 1;   // last visible key
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m_run = -INFINITY, l_run = 0.f;
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY;                   // running max in raw score units
+    float l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       if (!(ok = mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1, p.err))) break;
       tc_fence_after();
       float x[kBN];
+      {
+        uint32_t v[kBN / 32][32];
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(lane_base + (j & 1) * kBN + c * 32, v);
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(lane_base + (j & 1) * kBN + c * 32, v[c]);
         tc_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]);
+        for (int c = 0; c < kBN / 32; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[c][e]);
       }
       const int col0 = j * kBN;
+      if (col0 + kBN > full_keys) {   // tile reaches past some row's last visible key
+#pragma unroll
+        for (int e = 0; e < kBN; ++e)
+          if (col0 + e > p_row) x[e] = -INFINITY;
+      }
       float mt = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < kBN; ++e) {
-        x[e] = (col0 + e <= p_row) ? x[e] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, x[e]);
-      }
-      const float m_new = fmaxf(m_run, mt);
-      const float alpha = fast_exp2(m_run - m_new);
-      float rs = 0.f;
+      for (int e = 0; e < kBN; e += 2) mt = max3(mt, x[e], x[e + 1]);
+      // lazy rescale: move the max only when it grew by more than 2^kRescaleLog2
+      const bool grow = (mt - m_run) * sl2 > kRescaleLog2;
+      const float m_new = grow ? mt : m_run;
+      const float alpha = grow ? fast_exp2((m_run - m_new) * sl2) : 1.f;
+      const float nms = -m_new * sl2;
+      float rs0 = 0.f, rs1 = 0.f;
       uint32_t pk[kBN / 2];
 #pragma unroll
       for (int e = 0; e < kBN; e += 2) {
-        const float p0 = fast_exp2(x[e] - m_new), p1 = fast_exp2(x[e + 1] - m_new);
-        rs += p0 + p1;
+        float a0 = nms, a1 = nms;
+        ffma2(a0, a1, x[e], x[e + 1], sl2, sl2);
+        const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+        fadd2(rs0, rs1, p0, p1);
         pk[e / 2] = pack_bf16x2(p0, p1);
       }
-      l_run = l_run * alpha + rs;
-      // P buffer and O accumulator are free once the previous PV has finished
-      if (j > 0 && !(ok = mbar_wait_warp(o_done, (j - 1) & 1, p.err))) break;
-      tc_fence_after();
+      l_run = l_run * alpha + (rs0 + rs1);
+      // P buffer j%2 was last read by PV_{j-2}
+      if (j >= 2 && !(ok = mbar_wait_warp(&o_done[j & 1], ((j - 2) >> 1) & 1, p.err))) break;
+      uint8_t* pbuf = sP + (j & 1) * 2 * kChunkBytes;
 #pragma unroll
       for (int u = 0; u < kBN / 8; ++u) {
-        uint8_t* dst = sP + (u >> 3) * kChunkBytes + sw128(r, u & 7);
+        uint8_t* dst = pbuf + (u >> 3) * kChunkBytes + sw128(r, u & 7);
         *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       }
-      if (j > 0 && __any_sync(0xffffffffu, m_new > m_run)) {   // rescale O rows (running max grew; alpha = 1 elsewhere)
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // rescale O rows whose max moved (alpha = 1 elsewhere) once PV_{j-1} has landed
+        if (!(ok = mbar_wait_warp(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err))) break;
+        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -291,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // last tile reaches past the context: zero V rows >= Lk (they may hold
         // anything, and 0 * NaN would poison the PV product)
         const int s = j % kStages;
-        if (!(ok = mbar_wait_warp(&kv_full[s], (j / kStages) & 1, p.err))) break;
+        if (!(ok = mbar_wait_warp(&v_full[s], (j / kStages) & 1, p.err))) break;
         if (col0 + r >= Lk) {
 #pragma unroll
           for (int c = 0; c < kChunks; ++c)
@@ -303,9 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
     }
-    if (ok && nt > 0) ok = mbar_wait_warp(o_done, (nt - 1) & 1, p.err);
+    if (ok && nt > 0) ok = mbar_wait_warp(&o_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, p.err);
     tc_fence_after();
     if (ok) {   // warp-uniform: every lane takes part in the TMEM loads
       const float inv = 1.f / l_run;
