@@ -145,6 +145,37 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate.
+ * (The pages have no counterpart: this is a calling convenience of this
+ * library, not part of the method.)
+ *
+ * Some callers cannot give the library a device buffer of their own: a
+ * plugin inside a process that owns and pre-partitions all device memory, or
+ * a C caller with no handle on the allocator behind its device memory.  This
+ * entry point computes exactly what pa_decode computes, with the same
+ * arguments minus the workspace: the split-KV partials go to a fixed array
+ * of PA_DECODE_NOALLOC_SCRATCH_BYTES inside the library (reserved on every
+ * GPU that loads it, until the library is unloaded).  It allocates nothing.
+ *
+ * - Shapes whose pa_decode_workspace_size exceeds that limit are rejected
+ *   with PA_ERR_WORKSPACE before anything is launched (a larger
+ *   kv_chunk_size needs less scratch).
+ * - All calls on one device share the array: calls whose kernels may overlap
+ *   on that device race and return garbage, so order them.  The array keeps
+ *   the last call's contents; nothing needs it zeroed, since every partial a
+ *   call reads is written earlier in that call.
+ * - The array's device address is looked up on the first call made on each
+ *   device; make that first call before any stream capture starts.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                   const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs,
+                                   int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                   int32_t num_blocks, float scale, int32_t kv_chunk_size, void* stream);
+
+/*
  * pa_prefill_varlen -- varlen causal prefill against the paged cache.
  * ("Nano-vLLM 源碼學習" §二.2, prefill stage: varlen attention with prefix
  * cache support; "Architektur im Überblick", "Prefill- und

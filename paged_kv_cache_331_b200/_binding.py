@@ -31,6 +31,8 @@ _PROTOS = {
     "pa_prefill_varlen": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _i32, _i32, _i32,
                                          _i32, _i32, _i32, _f32, _i32, _vp]),
     "pa_device_error": (ctypes.c_int, [ctypes.POINTER(_i32), _vp]),
+    "pa_decode_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                         _f32, _i32, _vp]),
 }
 
 
@@ -128,6 +130,26 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len, sca
                                block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
                                int(max_context_len), B, hq, hkv, d, bs, nb, float(scale), int(kv_chunk_size), ws_ptr,
                                ws_len, _stream(q, stream)), "pa_decode")
+    return out
+
+
+def decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, *, out, kv_chunk_size=0,
+                   stream=None):
+    """pa_decode_noalloc: decode with the library's fixed split-KV scratch (no workspace, nothing allocated).
+
+    For callers that cannot provide device memory of their own; ``out`` must be given.  Calls that may run
+    concurrently on one GPU share the scratch and must be ordered."""
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("out", out)):
+        _cuda(t, n, torch.bfloat16); _dense(t, n)
+    _cuda(block_tables, "block_tables", torch.int32); _dense(block_tables, "block_tables")
+    _cuda(context_lens, "context_lens", torch.int32); _dense(context_lens, "context_lens")
+    B, hq, d = q.shape
+    nb, bs, hkv, _ = k_cache.shape
+    with torch.cuda.device(q.device):
+        _check(lib().pa_decode_noalloc(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                       block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+                                       int(max_context_len), B, hq, hkv, d, bs, nb, float(scale), int(kv_chunk_size),
+                                       _stream(q, stream)), "pa_decode_noalloc")
     return out
 
 
