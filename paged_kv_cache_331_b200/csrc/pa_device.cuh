@@ -114,6 +114,18 @@ __device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t nthreads
   return r != 0;
 }
 
+// Per-warpgroup register budget changes (all four warps of the warpgroup
+// execute them).  The sum over warpgroups must stay within the registers the
+// block was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ----------------------------------------------------------------------- TMA --
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {

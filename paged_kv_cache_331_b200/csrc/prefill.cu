@@ -14,7 +14,7 @@
 // Keys stream in tiles of 128 tokens gathered through the block table (TMA
 // boxes whose row coordinate is block_id * block_size + offset).
 //
-// Roles (320 threads):
+// Roles (384 threads):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r of a
 //              group owns row r (= TMEM lane r); it reads S from TMEM, masks,
 //              runs the online softmax in the exp2 domain (part of the
@@ -23,6 +23,8 @@
 //              the running max grows, and does the epilogue.
 //   warp 8     TMA producer: both Q tiles once, then K and V tiles in rings
 //              (K one tile ahead).
+//   warps 10-11 idle (they complete the third warpgroup, whose registers
+//              the softmax warpgroups borrow through setmaxnreg).
 //   warp 9     TMEM allocator and single-thread MMA issuer, in the order
 //              QK_A0 QK_B0 | PV_A0 QK_A1 PV_B0 QK_B1 | PV_A1 QK_A2 PV_B1 ...
 //              so that while one group runs its softmax the tensor core works
@@ -53,7 +55,13 @@ constexpr int kKStages = 2;         // K ring depth
 constexpr int kSoftmaxWarps = 8;    // two groups of four: tile A, tile B
 constexpr int kProducerWarp = kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+constexpr int kThreads = (kSoftmaxWarps + 4) * 32;   // third warpgroup: producer, MMA, two idle warps
+// Registers: the block launches with 168 per thread (384 x 168 = 64512); the
+// third warpgroup gives most of its share to the two softmax warpgroups:
+// 256 x 216 + 128 x 72 = 64512.
+constexpr uint32_t kSoftmaxRegs = 216;
+constexpr uint32_t kControlRegs = 72;
+static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= 384 * 168, "register split exceeds the launch budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kChunkBytes = kBM * 128;   // one 64-element-wide, 128-row swizzled chunk
 
@@ -244,7 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kProducerWarp) {
+  if (warp >= kSoftmaxWarps) {
+   regs_decrease<kControlRegs>();
+   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- producer --
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
@@ -299,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, v_issued - kVStages); j < v_issued; ++j)
         mbar_wait(&v_full[j % kVStages], (j / kVStages) & 1, p.err, kErrDrainTimeout);
     }
-  } else if (warp == kMmaWarp) {
+   } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       bool ok = mbar_wait(q_full, 0, p.err);
@@ -355,8 +365,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, p.err, kErrDrainTimeout);
     }
+   }   // warps 10-11: nothing to do
   } else {
     // ------------------------------------------------------------------ softmax --
+    regs_increase<kSoftmaxRegs>();
     const int x = warp >> 2;                   // 0: tile A, 1: tile B
     const int r = threadIdx.x & (kBM - 1);     // row / TMEM lane
     const int ntx = nt[x];
@@ -473,21 +485,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // hit distinct banks.
       const float inv = 1.f / l_run;
       uint8_t* srow = (x == 0 ? sK : sV) + r * (D * 2 + 16);
-      uint32_t v[D / 32][32];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + colO + c * 32, v[c]);
-      tc_wait_ld();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c)
+      for (int c = 0; c < D / 32; ++c) {   // 32 columns of O at a time
+        uint32_t v[32];
+        tmem_ld32(lane_base + colO + c * 32, v);
+        tc_wait_ld();
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(v[c][8 * u + 0]) * inv, __uint_as_float(v[c][8 * u + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(v[c][8 * u + 2]) * inv, __uint_as_float(v[c][8 * u + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(v[c][8 * u + 4]) * inv, __uint_as_float(v[c][8 * u + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(v[c][8 * u + 6]) * inv, __uint_as_float(v[c][8 * u + 7]) * inv);
+          w.x = pack_bf16x2(__uint_as_float(v[8 * u + 0]) * inv, __uint_as_float(v[8 * u + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(v[8 * u + 2]) * inv, __uint_as_float(v[8 * u + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(v[8 * u + 4]) * inv, __uint_as_float(v[8 * u + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(v[8 * u + 6]) * inv, __uint_as_float(v[8 * u + 7]) * inv);
           *reinterpret_cast<uint4*>(srow + (c * 4 + u) * 16) = w;
         }
+      }
       fence_proxy_async_smem();
       if (row_valid) {
         __nv_bfloat16* orow = p.out + (static_cast<int64_t>(q_row0 + i) * p.num_heads + g * G + hh) * D;
