@@ -7,8 +7,8 @@
 // start at num_cached_tokens, so query i of a sequence with Lk keys and Lq
 // new tokens sits at position Lk - Lq + i.)
 //
-// Work item = one CTA: two query tiles (A and B) of one (kv head g, sequence
-// b).  The M = 128 rows of a tile pack the G query heads that share kv head
+// Persistent: one CTA per SM walks a static list of work items; a work item
+// is two query tiles (A and B) of one (kv head g, sequence b).  The M = 128 rows of a tile pack the G query heads that share kv head
 // g, QP = 128 / G query positions each (row r -> head g*G + r / QP,
 // position qt*QP + r % QP), so every K/V tile loaded serves 2*G heads-tiles.
 // Keys stream in tiles of 128 tokens gathered through the block table (TMA
@@ -41,6 +41,7 @@
 // an error code, drains its copies and MMAs, frees TMEM and returns.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <math.h>
 
 #include "pa_device.cuh"
@@ -58,12 +59,20 @@ constexpr int kMmaWarp = kSoftmaxWarps + 1;
 constexpr int kThreads = (kSoftmaxWarps + 4) * 32;   // third warpgroup: producer, MMA, two idle warps
 // Registers: the block launches with 168 per thread (384 x 168 = 64512); the
 // third warpgroup gives most of its share to the two softmax warpgroups:
-// 256 x 216 + 128 x 72 = 64512.
-constexpr uint32_t kSoftmaxRegs = 216;
-constexpr uint32_t kControlRegs = 72;
+// 256 x 208 + 128 x 88 = 64512.
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kControlRegs = 88;
 static_assert(256 * kSoftmaxRegs + 128 * kControlRegs <= 384 * 168, "register split exceeds the launch budget");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kChunkBytes = kBM * 128;   // one 64-element-wide, 128-row swizzled chunk
+
+// Dynamic work distribution: each launch uses one of kSchedSlots counter
+// pairs {next item, CTAs finished}; CTAs take items with atomicAdd, and the
+// last CTA to finish puts both counters back to zero for the next launch that
+// uses the slot.  The host rotates slots between launches so that launches in
+// flight at the same time (on different streams) do not share one.
+constexpr int kSchedSlots = 64;
+__device__ unsigned int g_prefill_sched[kSchedSlots][2];
 
 struct PrefillParams {
   __nv_bfloat16* out;
@@ -77,6 +86,7 @@ struct PrefillParams {
   int32_t causal;
   float scale_log2;
   unsigned int* err;
+  int32_t sched_slot;
 };
 
 template <int D>
@@ -87,14 +97,14 @@ struct PrefillSmem {
   static constexpr size_t k_off = q_off + 2 * kChunks * kChunkBytes;
   static constexpr size_t v_off = k_off + kKStages * kChunks * kChunkBytes;
   static constexpr size_t bar_off = v_off + kVStages * kChunks * kChunkBytes;
-  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2], o_done[2], mma_done
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
+  // barriers: q_full, q_empty[2], k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2],
+  // o_done[2], mma_done, work_full[QN], work_empty[QN]
+  static constexpr int kWorkQ = 4;                      // work-item queue depth
+  static constexpr int kNumBars = 1 + 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1 + 2 * kWorkQ;
   static constexpr size_t tmem_slot_off = bar_off + kNumBars * 8;
-  static constexpr size_t bytes = tmem_slot_off + 16;
+  static constexpr size_t queue_off = tmem_slot_off + 16;
+  static constexpr size_t bytes = queue_off + kWorkQ * 4;
   static_assert(bytes <= 232448, "shared memory budget (227 KB per CTA)");
-  // epilogue staging: group A in the K ring, group B in the V ring, 128 rows of D*2+16 bytes
-  static_assert(kKStages * kChunks * kChunkBytes >= kBM * (D * 2 + 16), "staging A");
-  static_assert(kVStages * kChunks * kChunkBytes >= kBM * (D * 2 + 16), "staging B");
 };
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -149,13 +159,6 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float
 constexpr int kEmuEvery = 8;   // pairs k with k % kEmuEvery >= kEmuFrom are emulated
 constexpr int kEmuFrom = 5;
 
-__device__ __forceinline__ void bulk_store_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // A row's running max only moves when the tile max exceeds it by more than
 // 2^kRescaleLog2 (in exp2 units); until then the stale max keeps every
@@ -163,10 +166,54 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 // accumulator in TMEM needs no correction.
 constexpr float kRescaleLog2 = 8.0f;
 
+// One work item: a pair of query tiles (A = the later one, B) of one
+// (kv head, sequence).  Items are numbered pair-rank-major (rank 0 = the last
+// pair of each sequence, which sees the most keys), so consecutive items have
+// similar cost; each persistent CTA takes every gridDim.x-th item.
+struct Item {
+  int b, g;
+  int Lq, Lk, q_row0, pos_off;
+  bool valid, has_b;
+  int qtA, qtB, ntA, ntB, fullA, fullB;   // query tile, key tiles, keys every row sees
+};
+
+template <int QP>
+__device__ __forceinline__ Item decode_item(int t, int num_seqs, int num_kv_heads, const PrefillParams& p) {
+  Item it;
+  const int per_rank = num_seqs * num_kv_heads;
+  const int rank = t / per_rank;
+  it.b = (t % per_rank) / num_kv_heads;
+  it.g = t % num_kv_heads;
+  const int cq0 = __ldg(p.cu_seqlens_q);
+  const int cqb = __ldg(p.cu_seqlens_q + it.b);
+  it.Lq = __ldg(p.cu_seqlens_q + it.b + 1) - cqb;
+  it.Lk = __ldg(p.cu_seqlens_k + it.b + 1) - __ldg(p.cu_seqlens_k + it.b);
+  it.q_row0 = cqb - cq0;
+  it.pos_off = it.Lk - it.Lq;
+  const int ntq = (it.Lq + QP - 1) / QP;
+  const int npairs = (ntq + 1) / 2;
+  const int pair = npairs - 1 - rank;
+  it.valid = pair >= 0 && it.Lk >= it.Lq && it.Lk > 0;
+  it.has_b = it.valid && 2 * pair + 1 < ntq;
+  it.qtA = it.has_b ? 2 * pair + 1 : 2 * pair;
+  it.qtB = 2 * pair;
+  auto tiles = [&](int qt) {
+    const int i_last = min(it.Lq, (qt + 1) * QP) - 1;
+    const int n_keys = p.causal ? min(it.Lk, it.pos_off + i_last + 1) : it.Lk;
+    return it.valid ? (n_keys + kBN - 1) / kBN : 0;
+  };
+  it.ntA = tiles(it.qtA);
+  it.ntB = it.has_b ? tiles(it.qtB) : 0;
+  it.fullA = p.causal ? min(it.Lk, it.pos_off + it.qtA * QP + 1) : it.Lk;
+  it.fullB = p.causal ? min(it.Lk, it.pos_off + it.qtB * QP + 1) : it.Lk;
+  return it;
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tmV, const PrefillParams p, int32_t num_seqs,
+                   int32_t num_kv_heads, int32_t num_items) {
   using Smem = PrefillSmem<D>;
   constexpr int QP = kBM / G;                 // query positions per tile
   constexpr int kChunks = D / 64;
@@ -191,7 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + Smem::v_off;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::bar_off);
   uint64_t* q_full = bars;
-  uint64_t* k_full = q_full + 1;
+  uint64_t* q_empty = q_full + 1;            // [2]: Q_A, Q_B free again (their last QK has completed)
+  uint64_t* k_full = q_empty + 2;
   uint64_t* k_empty = k_full + kKStages;
   uint64_t* v_full = k_empty + kKStages;
   uint64_t* v_empty = v_full + kVStages;
@@ -199,34 +247,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + 2;             // [2]
   uint64_t* o_done = p_full + 2;             // [2]
   uint64_t* mma_done = o_done + 2;
+  uint64_t* work_full = mma_done + 1;        // [kWorkQ]: queue entry written (producer)
+  uint64_t* work_empty = work_full + Smem::kWorkQ;   // [kWorkQ]: entry read by the MMA thread and 8 softmax warps
+  int32_t* work_queue = reinterpret_cast<int32_t*>(smem + Smem::queue_off);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::tmem_slot_off);
+  constexpr int kWorkQ = Smem::kWorkQ;
 
-  const int b = blockIdx.z, g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cq0 = __ldg(p.cu_seqlens_q), cq_b = __ldg(p.cu_seqlens_q + b), cq_b1 = __ldg(p.cu_seqlens_q + b + 1);
-  const int Lq = cq_b1 - cq_b;
-  const int Lk = __ldg(p.cu_seqlens_k + b + 1) - __ldg(p.cu_seqlens_k + b);
-  const int ntq = (Lq + QP - 1) / QP;                     // query tiles of this sequence
-  const int npairs = (ntq + 1) / 2;
-  const int pair = npairs - 1 - static_cast<int>(blockIdx.x);   // longest pairs of a sequence first
-  if (pair < 0 || Lk < Lq || Lk <= 0) return;
-  // tile A is the later (longer) one of the pair; a pair of one tile has no B
-  const bool has_b = 2 * pair + 1 < ntq;
-  const int qt[2] = {has_b ? 2 * pair + 1 : 2 * pair, 2 * pair};
-  const int q_row0 = cq_b - cq0;                            // first q/out row of this sequence
-  const int pos_off = Lk - Lq;                              // position of query 0
-  int nt[2], full_keys[2];
-  for (int x = 0; x < 2; ++x) {
-    const int i_last = min(Lq, (qt[x] + 1) * QP) - 1;
-    const int n_keys = p.causal ? min(Lk, pos_off + i_last + 1) : Lk;
-    nt[x] = (n_keys + kBN - 1) / kBN;
-    full_keys[x] = p.causal ? min(Lk, pos_off + qt[x] * QP + 1) : Lk;   // keys every row of the tile sees
-  }
-  if (!has_b) nt[1] = 0;
-  const int ntA = nt[0], ntB = nt[1];        // ntB <= ntA
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(&q_empty[0], 1);
+    mbar_init(&q_empty[1], 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -241,6 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_done[x], 1);
     }
     mbar_init(mma_done, 1);
+    for (int q = 0; q < kWorkQ; ++q) {
+      mbar_init(&work_full[q], 1);
+      mbar_init(&work_empty[q], 1 + kSoftmaxWarps);
+    }
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -260,106 +296,163 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      const int ntiles_q = has_b ? 2 : 1;
-      mbar_arrive_expect_tx(q_full, ntiles_q * kChunks * kChunkBytes);
-      for (int x = 0; x < ntiles_q; ++x)
-        for (int hh = 0; hh < G; ++hh)
-          for (int c = 0; c < kChunks; ++c)
-            tma_load_3d(sQ + (x * kChunks + c) * kChunkBytes + hh * QP * 128, &tmQ, q_full, c * 64, g * G + hh,
-                        q_row0 + qt[x] * QP);
-      const int32_t* bt = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq;
       const int bs_shift = __ffs(p.block_size) - 1;
-      const int nblk_valid = (Lk + p.block_size - 1) >> bs_shift;
-      // One K or V tile: boxes past the last block of the sequence are skipped
-      // (their table entries may be -1).
-      auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int j) {
-        int nbox = kBN / p.box_rows;
-        while (nbox > 0 && ((j * kBN + (nbox - 1) * p.box_rows) >> bs_shift) >= nblk_valid) --nbox;
-        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox * p.box_rows * 128 * kChunks));
-        for (int k = 0; k < nbox; ++k) {
-          const int tok = j * kBN + k * p.box_rows;
-          const int blk = __ldg(bt + (tok >> bs_shift));
-          const int row = (blk << bs_shift) + (tok & (p.block_size - 1));
-          for (int c = 0; c < kChunks; ++c)
-            tma_load_3d(dst + c * kChunkBytes + k * p.box_rows * 128, map, bar, c * 64, g, row);
-        }
-      };
-      // K runs one tile ahead of V.
-      int k_issued = 0, v_issued = 0;
+      int kc = 0, vc = 0;            // K / V tiles issued so far (ring positions)
+      int qn[2] = {0, 0};            // Q tiles loaded so far per group
       bool ok = true;
-      if (ntA > 0 && (ok = mbar_wait(&k_empty[0], 1, p.err))) {
-        load_tile(&tmK, sK, &k_full[0], 0);
-        k_issued = 1;
-      }
-      for (int j = 0; ok && j < ntA; ++j) {
-        if (j + 1 < ntA) {
-          const int s1 = (j + 1) % kKStages;
-          if (!(ok = mbar_wait(&k_empty[s1], (((j + 1) / kKStages) & 1) ^ 1, p.err))) break;
-          load_tile(&tmK, sK + s1 * kChunks * kChunkBytes, &k_full[s1], j + 1);
-          k_issued = j + 2;
+      unsigned int* next_item = &g_prefill_sched[p.sched_slot][0];
+      for (int n = 0; ok; ++n) {
+        // take the next non-empty item and publish it to the MMA and softmax warps
+        int t;
+        Item it;
+        do {
+          t = static_cast<int>(atomicAdd(next_item, 1u));
+          if (t >= num_items) break;
+          it = decode_item<QP>(t, num_seqs, num_kv_heads, p);
+        } while (!it.valid);
+        const int q = n % kWorkQ;
+        if (!(ok = mbar_wait(&work_empty[q], ((n / kWorkQ) & 1) ^ 1, p.err))) break;
+        work_queue[q] = t < num_items ? t : -1;
+        mbar_arrive(&work_full[q]);   // release: the entry is visible to waiters of this phase
+        if (t >= num_items) break;
+        const int32_t* bt = p.block_tables + static_cast<int64_t>(it.b) * p.max_blocks_per_seq;
+        const int nblk_valid = (it.Lk + p.block_size - 1) >> bs_shift;
+        // One K or V tile: boxes past the last block of the sequence are skipped
+        // (their table entries may be -1).
+        auto load_tile = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* bar, int j) {
+          int nbox = kBN / p.box_rows;
+          while (nbox > 0 && ((j * kBN + (nbox - 1) * p.box_rows) >> bs_shift) >= nblk_valid) --nbox;
+          mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox * p.box_rows * 128 * kChunks));
+          for (int k = 0; k < nbox; ++k) {
+            const int tok = j * kBN + k * p.box_rows;
+            const int blk = __ldg(bt + (tok >> bs_shift));
+            const int row = (blk << bs_shift) + (tok & (p.block_size - 1));
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_3d(dst + c * kChunkBytes + k * p.box_rows * 128, map, bar, c * 64, it.g, row);
+          }
+        };
+        auto load_k = [&](int j) {
+          const int s = kc % kKStages;
+          if (!(ok = mbar_wait(&k_empty[s], ((kc / kKStages) & 1) ^ 1, p.err))) return;
+          load_tile(&tmK, sK + s * kChunks * kChunkBytes, &k_full[s], j);
+          ++kc;
+        };
+        auto load_v = [&](int j) {
+          const int s = vc % kVStages;
+          if (!(ok = mbar_wait(&v_empty[s], ((vc / kVStages) & 1) ^ 1, p.err))) return;
+          load_tile(&tmV, sV + s * kChunks * kChunkBytes, &v_full[s], j);
+          ++vc;
+        };
+        load_k(0);   // the first K tile goes ahead of Q: its slot may already be free
+        if (!ok) break;
+        const int nq = it.has_b ? 2 : 1;
+        for (int x = 0; ok && x < nq; ++x)
+          ok = mbar_wait(&q_empty[x], (qn[x] & 1) ^ 1, p.err);
+        if (!ok) break;
+        mbar_arrive_expect_tx(q_full, nq * kChunks * kChunkBytes);
+        for (int x = 0; x < nq; ++x) {
+          const int qt = x == 0 ? it.qtA : it.qtB;
+          for (int hh = 0; hh < G; ++hh)
+            for (int c = 0; c < kChunks; ++c)
+              tma_load_3d(sQ + (x * kChunks + c) * kChunkBytes + hh * QP * 128, &tmQ, q_full, c * 64,
+                          it.g * G + hh, it.q_row0 + qt * QP);
+          ++qn[x];
         }
-        const int s = j % kVStages;
-        if (!(ok = mbar_wait(&v_empty[s], ((j / kVStages) & 1) ^ 1, p.err))) break;
-        load_tile(&tmV, sV + s * kChunks * kChunkBytes, &v_full[s], j);
-        v_issued = j + 1;
+        for (int j = 0; ok && j < it.ntA; ++j) {   // K runs one tile ahead of V
+          if (j + 1 < it.ntA) load_k(j + 1);
+          if (ok) load_v(j);
+        }
       }
-      mbar_wait(q_full, 0, p.err, kErrDrainTimeout);
-      for (int j = max(0, k_issued - kKStages); j < k_issued; ++j)
-        mbar_wait(&k_full[j % kKStages], (j / kKStages) & 1, p.err, kErrDrainTimeout);
-      for (int j = max(0, v_issued - kVStages); j < v_issued; ++j)
-        mbar_wait(&v_full[j % kVStages], (j / kVStages) & 1, p.err, kErrDrainTimeout);
+      // never leave with copies in flight (time-limited; these have normally long landed)
+      for (int n = max(0, kc - kKStages); n < kc; ++n)
+        mbar_wait(&k_full[n % kKStages], (n / kKStages) & 1, p.err, kErrDrainTimeout);
+      for (int n = max(0, vc - kVStages); n < vc; ++n)
+        mbar_wait(&v_full[n % kVStages], (n / kVStages) & 1, p.err, kErrDrainTimeout);
+      const int items_q = qn[0];
+      if (items_q > 0) mbar_wait(q_full, (items_q - 1) & 1, p.err, kErrDrainTimeout);
     }
    } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- MMA issuer --
     if (lane == 0) {
-      bool ok = mbar_wait(q_full, 0, p.err);
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
-      auto issue_s = [&](int x, int j) {   // S_X = Q_X K_j^T
-        const int s = j % kKStages;
+      int kc = 0, vc = 0, nitems = 0;
+      int sx[2] = {0, 0};      // p_full waits so far per group
+      bool ok = true;
+      auto issue_s = [&](int x, int ks) {   // S_X = Q_X K^T, K from ring slot ks
 #pragma unroll
         for (int c = 0; c < kChunks; ++c)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = smem_desc(q_base + (x * kChunks + c) * kChunkBytes + kk * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(k_base + (s * kChunks + c) * kChunkBytes + kk * 32, 16, 1024, 2);
+            const uint64_t bd = smem_desc(k_base + (ks * kChunks + c) * kChunkBytes + kk * 32, 16, 1024, 2);
             tc_mma_ss(tmem + x * kBN, ad, bd, kIdescS, (c | kk) != 0);
           }
         tc_commit(&s_full[x]);
       };
-      auto issue_pv = [&](int x, int j) {   // O_X += P_X V_j, P_X from TMEM
-        const int s = j % kVStages;
+      auto issue_pv = [&](int x, int vs, bool first) {   // O_X (+)= P_X V, P_X from TMEM
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = smem_desc(v_base + s * kChunks * kChunkBytes + kk * 2048, kChunkBytes, 1024, 2);
-          tc_mma_ts(tmem + kColO + x * D, tmem + x * kBN + kk * 8, bd, kIdescO, (j | kk) != 0);
+          const uint64_t bd = smem_desc(v_base + vs * kChunks * kChunkBytes + kk * 2048, kChunkBytes, 1024, 2);
+          tc_mma_ts(tmem + kColO + x * D, tmem + x * kBN + kk * 8, bd, kIdescO, !(first && kk == 0));
         }
         tc_commit(&o_done[x]);
       };
-      if (ok && ntA > 0 && (ok = mbar_wait(&k_full[0], 0, p.err))) {
-        tc_fence_after();
-        issue_s(0, 0);
-        if (ntB > 0) issue_s(1, 0);
-        tc_commit(&k_empty[0]);
-      }
-      for (int j = 0; ok && j < ntA; ++j) {
-        const int sv = j % kVStages;
-        if (!(ok = mbar_wait(&v_full[sv], (j / kVStages) & 1, p.err))) break;
-        const bool more = j + 1 < ntA;
-        if (more && !(ok = mbar_wait(&k_full[(j + 1) % kKStages], ((j + 1) / kKStages) & 1, p.err))) break;
-        // tile A
-        if (!(ok = mbar_wait(&p_full[0], j & 1, p.err))) break;
-        tc_fence_after();
-        issue_pv(0, j);
-        if (more) issue_s(0, j + 1);
-        // tile B
-        if (j < ntB) {
-          if (!(ok = mbar_wait(&p_full[1], j & 1, p.err))) break;
+      for (int n = 0; ok; ++n) {
+        const int q = n % kWorkQ;
+        if (!(ok = mbar_wait(&work_full[q], (n / kWorkQ) & 1, p.err))) break;
+        const int t = work_queue[q];
+        mbar_arrive(&work_empty[q]);
+        if (t < 0) break;
+        const Item it = decode_item<QP>(t, num_seqs, num_kv_heads, p);
+        const int ntA = it.ntA, ntB = it.ntB;
+        if (!(ok = mbar_wait(q_full, nitems & 1, p.err))) break;
+        ++nitems;
+        {
+          const int ks = kc % kKStages;
+          if (!(ok = mbar_wait(&k_full[ks], (kc / kKStages) & 1, p.err))) break;
           tc_fence_after();
-          issue_pv(1, j);
-          if (j + 1 < ntB) issue_s(1, j + 1);
+          issue_s(0, ks);
+          if (ntA == 1) tc_commit(&q_empty[0]);
+          if (ntB > 0) {
+            issue_s(1, ks);
+            if (ntB == 1) tc_commit(&q_empty[1]);
+          }
+          tc_commit(&k_empty[ks]);
+          ++kc;
         }
-        tc_commit(&v_empty[sv]);
-        if (more) tc_commit(&k_empty[(j + 1) % kKStages]);
+        for (int j = 0; ok && j < ntA; ++j) {
+          const int vs = vc % kVStages;
+          if (!(ok = mbar_wait(&v_full[vs], (vc / kVStages) & 1, p.err))) break;
+          const bool more = j + 1 < ntA;
+          const int ks = kc % kKStages;
+          if (more && !(ok = mbar_wait(&k_full[ks], (kc / kKStages) & 1, p.err))) break;
+          // tile A
+          if (!(ok = mbar_wait(&p_full[0], sx[0] & 1, p.err))) break;
+          ++sx[0];
+          tc_fence_after();
+          issue_pv(0, vs, j == 0);
+          if (more) {
+            issue_s(0, ks);
+            if (j + 2 == ntA) tc_commit(&q_empty[0]);
+          }
+          // tile B
+          if (j < ntB) {
+            if (!(ok = mbar_wait(&p_full[1], sx[1] & 1, p.err))) break;
+            ++sx[1];
+            tc_fence_after();
+            issue_pv(1, vs, j == 0);
+            if (j + 1 < ntB) {
+              issue_s(1, ks);
+              if (j + 2 == ntB) tc_commit(&q_empty[1]);
+            }
+          }
+          tc_commit(&v_empty[vs]);
+          ++vc;
+          if (more) {
+            tc_commit(&k_empty[ks]);
+            ++kc;
+          }
+        }
       }
       // wait for every MMA this thread issued before TMEM can be released
       tc_commit(mma_done);
@@ -371,122 +464,132 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_increase<kSoftmaxRegs>();
     const int x = warp >> 2;                   // 0: tile A, 1: tile B
     const int r = threadIdx.x & (kBM - 1);     // row / TMEM lane
-    const int ntx = nt[x];
-    const int hh = r / QP;
-    const int i = qt[x] * QP + (r % QP);       // query index within the sequence
-    const bool row_valid = i < Lq && (x == 0 || has_b);
-    const int p_row = p.causal ? min(pos_off + i, Lk - 1) : Lk - 1;   // last visible key
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t colS = x * kBN, colO = kColO + x * D;
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;                   // running max in raw score units
-    float l_run = 0.f;
+    int ns = 0;                  // S tiles consumed so far (s_full phases)
+    int no = 0;                  // PVs of this group issued so far (o_done phases)
     bool ok = true;
-    for (int j = 0; j < ntx; ++j) {
-      // S_X(j) complete implies PV_X(j-1) complete: P columns and O are free
-      if (!(ok = mbar_wait_warp(&s_full[x], j & 1, p.err))) break;
-      tc_fence_after();
-      float xs[kBN];
-      {
-        uint32_t v[kBN / 32][32];
+    for (int n = 0; ok; ++n) {
+      const int q = n % kWorkQ;
+      if (!(ok = mbar_wait_warp(&work_full[q], (n / kWorkQ) & 1, p.err))) break;
+      const int t = work_queue[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&work_empty[q]);
+      if (t < 0) break;
+      const Item it = decode_item<QP>(t, num_seqs, num_kv_heads, p);
+      const int ntx = x == 0 ? it.ntA : it.ntB;
+      if (ntx == 0) continue;
+      const int full_keys = x == 0 ? it.fullA : it.fullB;
+      const int hh = r / QP;
+      const int i = (x == 0 ? it.qtA : it.qtB) * QP + (r % QP);  // query index within the sequence
+      const bool row_valid = i < it.Lq;
+      const int p_row = p.causal ? min(it.pos_off + i, it.Lk - 1) : it.Lk - 1;   // last visible key
+      float m_run = -INFINITY;                 // running max in raw score units
+      float l_run = 0.f;
+      for (int j = 0; j < ntx; ++j) {
+        // S_X(j) complete implies PV_X(j-1) complete: P columns and O are free
+        if (!(ok = mbar_wait_warp(&s_full[x], ns & 1, p.err))) break;
+        ++ns;
+        tc_fence_after();
+        float xs[kBN];
+        {
+          uint32_t v[kBN / 32][32];
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(lane_base + colS + c * 32, v[c]);
-        tc_wait_ld();
-#pragma unroll
-        for (int c = 0; c < kBN / 32; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) xs[c * 32 + e] = __uint_as_float(v[c][e]);
-      }
-      const int col0 = j * kBN;
-      if (col0 + kBN > full_keys[x]) {   // tile reaches past some row's last visible key
-#pragma unroll
-        for (int e = 0; e < kBN; ++e)
-          if (col0 + e > p_row) xs[e] = -INFINITY;
-      }
-      float mx8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(xs[u], xs[u + 8]);
-#pragma unroll
-      for (int e = 16; e < kBN; e += 16)
-#pragma unroll
-        for (int u = 0; u < 8; u += 2) {
-          mx8[u] = max3(mx8[u], xs[e + u], xs[e + u + 8]);
-          mx8[u + 1] = max3(mx8[u + 1], xs[e + u + 1], xs[e + u + 9]);
-        }
-      const float mt = fmaxf(fmaxf(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5])), fmaxf(mx8[6], mx8[7]));
-      // lazy rescale: move the max only when it grew by more than 2^kRescaleLog2
-      const bool grow = (mt - m_run) * sl2 > kRescaleLog2;
-      const float m_new = grow ? mt : m_run;
-      const float alpha = grow ? fast_exp2((m_run - m_new) * sl2) : 1.f;
-      const float nms = -m_new * sl2;
-      float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[kBN / 2];
-#pragma unroll
-      for (int e = 0; e < kBN; e += 2) {
-        float a0 = nms, a1 = nms;
-        ffma2(a0, a1, xs[e], xs[e + 1], sl2, sl2);
-        float p0, p1;
-        if ((e / 2) % kEmuEvery >= kEmuFrom) {
-          exp2_poly2(p0, p1, a0, a1);
-        } else {
-          p0 = fast_exp2(a0);
-          p1 = fast_exp2(a1);
-        }
-        const int k = (e / 2) & 3;
-        fadd2(rs[2 * k], rs[2 * k + 1], p0, p1);
-        pk[e / 2] = pack_bf16x2(p0, p1);
-      }
-      l_run = l_run * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
-      tmem_st32(lane_base + colS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(lane_base + colS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // rescale O rows whose max moved (alpha = 1 elsewhere)
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + colO + c * 32, v);
+          for (int c = 0; c < kBN / 32; ++c) tmem_ld32(lane_base + colS + c * 32, v[c]);
           tc_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-          tmem_st32(lane_base + colO + c * 32, v);
-        }
-      }
-      tc_wait_st();
-      m_run = m_new;
-      if (x == 0 && col0 + kBN > Lk) {
-        // the last tile reaches past the context: zero V rows >= Lk before any
-        // PV reads them (group A's PV of this tile comes first; 0 * NaN would
-        // poison the product)
-        const int s = j % kVStages;
-        if (!(ok = mbar_wait_warp(&v_full[s], (j / kVStages) & 1, p.err))) break;
-        if (col0 + r >= Lk) {
+          for (int c = 0; c < kBN / 32; ++c)
 #pragma unroll
-          for (int c = 0; c < kChunks; ++c)
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              *reinterpret_cast<uint4*>(sV + (s * kChunks + c) * kChunkBytes + r * 128 + u * 16) =
-                  make_uint4(0, 0, 0, 0);
+            for (int e = 0; e < 32; ++e) xs[c * 32 + e] = __uint_as_float(v[c][e]);
         }
-        fence_proxy_async_smem();
+        const int col0 = j * kBN;
+        if (col0 + kBN > full_keys) {   // tile reaches past some row's last visible key
+#pragma unroll
+          for (int e = 0; e < kBN; ++e)
+            if (col0 + e > p_row) xs[e] = -INFINITY;
+        }
+        float mx8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(xs[u], xs[u + 8]);
+#pragma unroll
+        for (int e = 16; e < kBN; e += 16)
+#pragma unroll
+          for (int u = 0; u < 8; u += 2) {
+            mx8[u] = max3(mx8[u], xs[e + u], xs[e + u + 8]);
+            mx8[u + 1] = max3(mx8[u + 1], xs[e + u + 1], xs[e + u + 9]);
+          }
+        const float mt =
+            fmaxf(fmaxf(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5])), fmaxf(mx8[6], mx8[7]));
+        // lazy rescale: move the max only when it grew by more than 2^kRescaleLog2
+        const bool grow = (mt - m_run) * sl2 > kRescaleLog2;
+        const float m_new = grow ? mt : m_run;
+        const float alpha = grow ? fast_exp2((m_run - m_new) * sl2) : 1.f;
+        const float nms = -m_new * sl2;
+        float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[kBN / 2];
+#pragma unroll
+        for (int e = 0; e < kBN; e += 2) {
+          float a0 = nms, a1 = nms;
+          ffma2(a0, a1, xs[e], xs[e + 1], sl2, sl2);
+          float p0, p1;
+          if ((e / 2) % kEmuEvery >= kEmuFrom) {
+            exp2_poly2(p0, p1, a0, a1);
+          } else {
+            p0 = fast_exp2(a0);
+            p1 = fast_exp2(a1);
+          }
+          const int k = (e / 2) & 3;
+          fadd2(rs[2 * k], rs[2 * k + 1], p0, p1);
+          pk[e / 2] = pack_bf16x2(p0, p1);
+        }
+        l_run = l_run * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
+        tmem_st32(lane_base + colS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(lane_base + colS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // rescale O rows whose max moved (alpha = 1 elsewhere)
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(lane_base + colO + c * 32, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            tmem_st32(lane_base + colO + c * 32, v);
+          }
+        }
+        tc_wait_st();
+        m_run = m_new;
+        if (x == 0 && col0 + kBN > it.Lk) {
+          // the last tile reaches past the context: zero V rows >= Lk before any
+          // PV reads them (group A's PV of this tile comes first; 0 * NaN would
+          // poison the product).  This tile's V slot is the one the MMA warp
+          // consumes for tile j of this item.
+          const int vs = (no + j) % kVStages;
+          if (!(ok = mbar_wait_warp(&v_full[vs], ((no + j) / kVStages) & 1, p.err))) break;
+          if (col0 + r >= it.Lk) {
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+              for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4*>(sV + (vs * kChunks + c) * kChunkBytes + r * 128 + u * 16) =
+                    make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive(&p_full[x]);
       }
-      tc_fence_before();
-      mbar_arrive(&p_full[x]);
-    }
-    if (ok && ntx > 0) ok = mbar_wait_warp(&o_done[x], (ntx - 1) & 1, p.err);
-    // Group B stages its rows in the V ring, which tile A's remaining PVs may
-    // still read when B has fewer key tiles: wait for every MMA of the CTA.
-    if (ok && ntx > 0 && x == 1) ok = mbar_wait_warp(mma_done, 0, p.err);
-    tc_fence_after();
-    if (ok && ntx > 0) {   // warp-uniform: every lane takes part in the TMEM loads
-      // O row -> bf16 -> shared memory, then one bulk copy per valid row to its
-      // place in out.  Group A stages in the K ring (every QK has completed once
-      // PV_A of the last tile has), group B in the V ring (after every MMA of
-      // the CTA).  Rows are padded by 16 bytes so the 16-byte writes of a warp
-      // hit distinct banks.
+      if (!ok) break;
+      no += ntx;
+      ok = mbar_wait_warp(&o_done[x], (no - 1) & 1, p.err);
+      if (!ok) break;
+      tc_fence_after();
+      // Epilogue: O row -> bf16 -> out (16-byte stores of this thread's row).
       const float inv = 1.f / l_run;
-      uint8_t* srow = (x == 0 ? sK : sV) + r * (D * 2 + 16);
+      __nv_bfloat16* orow = p.out + (static_cast<int64_t>(it.q_row0 + i) * p.num_heads + it.g * G + hh) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {   // 32 columns of O at a time
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(lane_base + colO + c * 32, v);
         tc_wait_ld();
@@ -497,27 +600,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.y = pack_bf16x2(__uint_as_float(v[8 * u + 2]) * inv, __uint_as_float(v[8 * u + 3]) * inv);
           w.z = pack_bf16x2(__uint_as_float(v[8 * u + 4]) * inv, __uint_as_float(v[8 * u + 5]) * inv);
           w.w = pack_bf16x2(__uint_as_float(v[8 * u + 6]) * inv, __uint_as_float(v[8 * u + 7]) * inv);
-          *reinterpret_cast<uint4*>(srow + (c * 4 + u) * 16) = w;
+          if (row_valid) *reinterpret_cast<uint4*>(orow + c * 32 + u * 8) = w;
         }
       }
-      fence_proxy_async_smem();
-      if (row_valid) {
-        __nv_bfloat16* orow = p.out + (static_cast<int64_t>(q_row0 + i) * p.num_heads + g * G + hh) * D;
-        bulk_store_s2g(orow, srow, D * 2);
-        bulk_commit();
-        bulk_wait_read();
-      }
+      tc_fence_before();     // TMEM reads of O done before the next item's PV_X(0) may overwrite it
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  if (threadIdx.x == 0) {
+    // the last CTA of the launch returns the scheduling slot to zero
+    __threadfence();
+    if (atomicAdd(&g_prefill_sched[p.sched_slot][1], 1u) == gridDim.x - 1) {
+      g_prefill_sched[p.sched_slot][0] = 0;
+      g_prefill_sched[p.sched_slot][1] = 0;
+      __threadfence();
+    }
+  }
 }
 
 template <int D, int G>
 pa_status launch_typed(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                       const PrefillParams& p, dim3 grid, cudaStream_t stream) {
+                       const PrefillParams& p, dim3 grid, int32_t num_seqs, int32_t num_kv_heads, int32_t num_items,
+                       cudaStream_t stream) {
   using Smem = PrefillSmem<D>;
   static int configured_device = -1;
   const DeviceInfo* di = current_device_info();
@@ -530,7 +637,7 @@ pa_status launch_typed(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUt
     }
     configured_device = di->device;
   }
-  prefill_kernel<D, G><<<grid, kThreads, Smem::bytes, stream>>>(tmQ, tmK, tmV, p);
+  prefill_kernel<D, G><<<grid, kThreads, Smem::bytes, stream>>>(tmQ, tmK, tmV, p, num_seqs, num_kv_heads, num_items);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("prefill launch: %s", cudaGetErrorString(e));
@@ -541,12 +648,12 @@ pa_status launch_typed(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUt
 
 template <int D>
 pa_status dispatch_group(int G, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                         const PrefillParams& p, dim3 grid, cudaStream_t stream) {
+                         const PrefillParams& p, dim3 grid, int32_t ns, int32_t nkv, int32_t ni, cudaStream_t stream) {
   switch (G) {
-    case 1: return launch_typed<D, 1>(tmQ, tmK, tmV, p, grid, stream);
-    case 2: return launch_typed<D, 2>(tmQ, tmK, tmV, p, grid, stream);
-    case 4: return launch_typed<D, 4>(tmQ, tmK, tmV, p, grid, stream);
-    case 8: return launch_typed<D, 8>(tmQ, tmK, tmV, p, grid, stream);
+    case 1: return launch_typed<D, 1>(tmQ, tmK, tmV, p, grid, ns, nkv, ni, stream);
+    case 2: return launch_typed<D, 2>(tmQ, tmK, tmV, p, grid, ns, nkv, ni, stream);
+    case 4: return launch_typed<D, 4>(tmQ, tmK, tmV, p, grid, ns, nkv, ni, stream);
+    case 8: return launch_typed<D, 8>(tmQ, tmK, tmV, p, grid, ns, nkv, ni, stream);
     default: break;
   }
   set_last_error("prefill: query heads per kv head = %d not supported", G);
@@ -581,11 +688,20 @@ pa_status launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
   p.causal = a.causal ? 1 : 0;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.err = current_device_info()->error_word;
+  static std::atomic<uint32_t> launches{0};
+  p.sched_slot = static_cast<int32_t>(launches.fetch_add(1) % kSchedSlots);
+  // persistent grid: at most one CTA per SM, each walking every gridDim.x-th work item
   const int max_tiles = (a.max_seqlen_q + QP - 1) / QP;
-  const dim3 grid(static_cast<unsigned>((max_tiles + 1) / 2), static_cast<unsigned>(a.num_kv_heads),
-                  static_cast<unsigned>(a.num_seqs));
-  return a.head_dim == 128 ? dispatch_group<128>(G, tmQ, tmK, tmV, p, grid, stream)
-                           : dispatch_group<64>(G, tmQ, tmK, tmV, p, grid, stream);
+  const int64_t items64 = static_cast<int64_t>((max_tiles + 1) / 2) * a.num_kv_heads * a.num_seqs;
+  if (items64 > INT32_MAX) {
+    set_last_error("prefill: too many work items");
+    return PA_ERR_UNSUPPORTED;
+  }
+  const int32_t items = static_cast<int32_t>(items64);
+  const int sms = current_device_info()->sm_count;
+  const dim3 grid(static_cast<unsigned>(items < sms ? items : sms));
+  return a.head_dim == 128 ? dispatch_group<128>(G, tmQ, tmK, tmV, p, grid, a.num_seqs, a.num_kv_heads, items, stream)
+                           : dispatch_group<64>(G, tmQ, tmK, tmV, p, grid, a.num_seqs, a.num_kv_heads, items, stream);
 }
 
 }  // namespace pa
