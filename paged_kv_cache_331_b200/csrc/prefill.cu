@@ -157,7 +157,7 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float
 
 // Every kEmuEvery-th pair of softmax exponentials uses exp2_poly2.
 constexpr int kEmuEvery = 8;   // pairs k with k % kEmuEvery >= kEmuFrom are emulated
-constexpr int kEmuFrom = 5;
+constexpr int kEmuFrom = 6;
 
 
 // A row's running max only moves when the tile max exceeds it by more than
@@ -378,23 +378,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       int kc = 0, vc = 0, nitems = 0;
       int sx[2] = {0, 0};      // p_full waits so far per group
       bool ok = true;
+      // Descriptors differ only in their start-address field (bits 0-13, in
+      // 16-byte units): build one base per operand and add offsets.
+      const uint64_t q_desc = smem_desc(q_base, 16, 1024, 2);
+      const uint64_t k_desc = smem_desc(k_base, 16, 1024, 2);
+      const uint64_t v_desc = smem_desc(v_base, kChunkBytes, 1024, 2);
       auto issue_s = [&](int x, int ks) {   // S_X = Q_X K^T, K from ring slot ks
+        const uint64_t qa = q_desc + ((x * kChunks * kChunkBytes) >> 4);
+        const uint64_t kb = k_desc + ((ks * kChunks * kChunkBytes) >> 4);
 #pragma unroll
         for (int c = 0; c < kChunks; ++c)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc(q_base + (x * kChunks + c) * kChunkBytes + kk * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(k_base + (ks * kChunks + c) * kChunkBytes + kk * 32, 16, 1024, 2);
-            tc_mma_ss(tmem + x * kBN, ad, bd, kIdescS, (c | kk) != 0);
+            const uint32_t off = (c * kChunkBytes + kk * 32) >> 4;
+            tc_mma_ss(tmem + x * kBN, qa + off, kb + off, kIdescS, (c | kk) != 0);
           }
         tc_commit(&s_full[x]);
       };
       auto issue_pv = [&](int x, int vs, bool first) {   // O_X (+)= P_X V, P_X from TMEM
+        const uint64_t vb = v_desc + ((vs * kChunks * kChunkBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = smem_desc(v_base + vs * kChunks * kChunkBytes + kk * 2048, kChunkBytes, 1024, 2);
-          tc_mma_ts(tmem + kColO + x * D, tmem + x * kBN + kk * 8, bd, kIdescO, !(first && kk == 0));
-        }
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          tc_mma_ts(tmem + kColO + x * D, tmem + x * kBN + kk * 8, vb + ((kk * 2048) >> 4), kIdescO,
+                    !(first && kk == 0));
         tc_commit(&o_done[x]);
       };
       for (int n = 0; ok; ++n) {
