@@ -87,6 +87,7 @@ struct PrefillParams {
   float scale_log2;
   unsigned int* err;
   int32_t sched_slot;
+  int32_t out_v8;            // out is 32-byte aligned: write 32-byte vectors
 };
 
 template <int D>
@@ -599,14 +600,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t v[32];
         tmem_ld32(lane_base + colO + c * 32, v);
         tc_wait_ld();
+        uint32_t w[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(v[8 * u + 0]) * inv, __uint_as_float(v[8 * u + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(v[8 * u + 2]) * inv, __uint_as_float(v[8 * u + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(v[8 * u + 4]) * inv, __uint_as_float(v[8 * u + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(v[8 * u + 6]) * inv, __uint_as_float(v[8 * u + 7]) * inv);
-          if (row_valid) *reinterpret_cast<uint4*>(orow + c * 32 + u * 8) = w;
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
+        if (row_valid) {
+          if (p.out_v8) {   // full 32-byte sectors: half the store transactions of 16-byte vectors
+            st_v8(orow + c * 32, *reinterpret_cast<const uint32_t(*)[8]>(&w[0]));
+            st_v8(orow + c * 32 + 16, *reinterpret_cast<const uint32_t(*)[8]>(&w[8]));
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              *reinterpret_cast<uint4*>(orow + c * 32 + u * 8) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          }
         }
       }
       tc_fence_before();     // TMEM reads of O done before the next item's PV_X(0) may overwrite it
@@ -694,6 +700,7 @@ pa_status launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
   p.causal = a.causal ? 1 : 0;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.err = current_device_info()->error_word;
+  p.out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
   static std::atomic<uint32_t> launches{0};
   p.sched_slot = static_cast<int32_t>(launches.fetch_add(1) % kSchedSlots);
   // persistent grid: at most one CTA per SM, each walking every gridDim.x-th work item
