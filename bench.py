@@ -368,6 +368,58 @@ def bench_prefill(args, dev, peaks):
     }
 
 
+def bench_graph(args, dev):
+    """Store + decode of one layer at small batches, eager against a replayed CUDA graph (the engine's decode
+    graphs): each step ends with a host synchronisation, as a token-by-token loop does, so the time includes
+    the host's launch latency that the graph removes."""
+    import torch
+    import paged_kv_cache_331_b200 as pa
+    from paged_kv_cache_331_b200 import workloads as W
+    from paged_kv_cache_331_b200.graphs import DecodeGraphRunner
+
+    res = {}
+    for bs in (1, 8, 32):
+        rng = np.random.default_rng(60 + bs)
+        w = W.decode_workload(np.full(bs, 1024, np.int32), 16, 8, 128, 256, rng=rng)
+        q, kc, vc = to_dev(w.q, "bf16", dev), to_dev(w.k_cache, "bf16", dev), to_dev(w.v_cache, "bf16", dev)
+        nk, nv = to_dev(w.new_k, "bf16", dev), to_dev(w.new_v, "bf16", dev)
+        slots, bt, cl = (to_dev(w.slot_mapping, "i32", dev), to_dev(w.block_tables, "i32", dev),
+                         to_dev(w.context_lens, "i32", dev))
+        out = torch.empty_like(q)
+        ws = torch.empty(max(16, pa.decode_workspace_size(bs, 16, 8, 128, 1024, 256, 0)), dtype=torch.uint8,
+                         device=dev)
+        runner = DecodeGraphRunner(kc, vc, 16, max_bs=bs, max_blocks_per_seq=bt.shape[1], max_context_len=1024,
+                                   scale=w.scale)
+        pbs = runner.load(q, nk, nv, slots, bt, cl)
+
+        def eager():
+            pa.store_kvcache(nk, nv, kc, vc, slots)
+            pa.decode(q, kc, vc, bt, cl, 1024, w.scale, out=out, workspace=ws)
+
+        def graph():
+            runner.replay(pbs)
+
+        times = {}
+        for name, fn in (("eager", eager), ("graph", graph)):
+            for _ in range(5):
+                fn()
+            torch.cuda.synchronize(dev)
+            n = max(20, min(args.steps, 300))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(n):
+                fn()
+                torch.cuda.current_stream(dev).synchronize()
+            b.record()
+            torch.cuda.synchronize(dev)
+            times[name] = a.elapsed_time(b) / n * 1e3
+        assert torch.equal(out.view(torch.int16), runner.out[:bs].view(torch.int16))
+        res[str(bs)] = {"eager_us": round(times["eager"], 2), "graph_us": round(times["graph"], 2)}
+    assert pa.device_error() == 0
+    return {"step": "store_kvcache + decode, context 1024, 16 q / 8 kv heads, D 128, host sync per step",
+            "per_batch": res}
+
+
 def cpu_baseline(w, budget_s=12.0):
     """The oracle as it stands, on this host's cores: store + decode of the same workload, repeated for about
     budget_s seconds."""
@@ -376,7 +428,7 @@ def cpu_baseline(w, budget_s=12.0):
     kc, vc = w.k_cache.copy(), w.v_cache.copy()
     kv_bytes, _ = decode_algorithmic_bytes(w)
     reps, t_total = 0, 0.0
-    while t_total < budget_s and reps < 50:
+    while t_total < budget_s and reps < 1000:
         t = time.perf_counter()
         orc.store_kvcache(w.new_k, w.new_v, kc, vc, w.slot_mapping)
         orc.decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale)
@@ -395,6 +447,7 @@ def run_ours(args, world, rank, local):
     pa.lib()
     w, d = bench_decode(args, world, rank, dev, peaks)
     pre = bench_prefill(args, dev, peaks) if (rank == 0 and not args.no_prefill) else None
+    gr = bench_graph(args, dev) if (rank == 0 and not args.no_graph) else None
     cpu = cpu_baseline(w) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if rank != 0:
         return
@@ -422,6 +475,8 @@ def run_ours(args, world, rank, local):
     }
     if pre is not None:
         line["prefill"] = pre
+    if gr is not None:
+        line["graph"] = gr
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
@@ -484,6 +539,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

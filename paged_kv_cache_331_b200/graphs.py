@@ -1,0 +1,112 @@
+"""CUDA-graph capture of the decode step (store_kvcache + decode).
+
+"Architektur im Überblick", section "CUDA Graph Optimierung": the engine
+captures its decode step once per batch size in [1, 2, 4, 8] + [16, 32, ...,
+max_bs], in descending order and into one shared memory pool, and replays
+the smallest captured graph that holds the current batch.  This runner does
+the same for the attention step of one layer: the new tokens' K/V rows are
+scattered into the cache and every sequence attends over its blocks.
+
+Rows past the real batch are padding: their slot is -1 (the store skips them)
+and their context length 0 (decode writes zeros), so a padded replay computes
+exactly what an unpadded call computes for the real rows.  The KV cache, the
+static input buffers and the decode workspace keep their addresses for the
+runner's lifetime: the captured kernels (and their TMA tensor maps) refer to
+them.  Every step of the computation is a kernel of libpagedattn.so; torch
+supplies the graph objects, buffers and streams.
+"""
+from __future__ import annotations
+
+import bisect
+
+import torch
+
+from . import _binding as pa
+
+
+def graph_batch_sizes(max_bs: int):
+    """[1, 2, 4, 8] + [16, 32, ..., max_bs] (sizes above max_bs dropped)."""
+    return [b for b in [1, 2, 4, 8] + list(range(16, max_bs + 1, 16)) if b <= max_bs]
+
+
+class DecodeGraphRunner:
+    """Captured store_kvcache + decode steps for one layer's paged KV cache."""
+
+    def __init__(self, k_cache, v_cache, num_heads, max_bs, max_blocks_per_seq, max_context_len, scale,
+                 kv_chunk_size=0):
+        if not (k_cache.is_cuda and v_cache.is_cuda):
+            raise TypeError("the KV cache must live on a CUDA device")
+        self.k_cache, self.v_cache = k_cache, v_cache
+        nb, bs_blk, hkv, d = k_cache.shape
+        self.num_heads, self.num_kv_heads, self.head_dim, self.block_size = num_heads, hkv, d, bs_blk
+        self.max_bs, self.max_blocks_per_seq = max_bs, max_blocks_per_seq
+        self.max_context_len, self.scale, self.kv_chunk_size = max_context_len, scale, kv_chunk_size
+        dev = k_cache.device
+        bf = torch.bfloat16
+        self.q = torch.zeros(max_bs, num_heads, d, dtype=bf, device=dev)
+        self.new_k = torch.zeros(max_bs, hkv, d, dtype=bf, device=dev)
+        self.new_v = torch.zeros(max_bs, hkv, d, dtype=bf, device=dev)
+        self.slot_mapping = torch.full((max_bs,), -1, dtype=torch.int32, device=dev)
+        self.block_tables = torch.full((max_bs, max_blocks_per_seq), -1, dtype=torch.int32, device=dev)
+        self.context_lens = torch.zeros(max_bs, dtype=torch.int32, device=dev)
+        self.out = torch.zeros(max_bs, num_heads, d, dtype=bf, device=dev)
+        self.graph_bs = graph_batch_sizes(max_bs)
+        ws = max(pa.decode_workspace_size(b, num_heads, hkv, d, max_context_len, bs_blk, kv_chunk_size)
+                 for b in self.graph_bs)
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+        self.graphs = {}
+        self._capture()
+
+    def _step(self, bs):
+        pa.store_kvcache(self.new_k[:bs], self.new_v[:bs], self.k_cache, self.v_cache, self.slot_mapping[:bs])
+        pa.decode(self.q[:bs], self.k_cache, self.v_cache, self.block_tables[:bs], self.context_lens[:bs],
+                  self.max_context_len, self.scale, out=self.out[:bs], workspace=self.workspace,
+                  kv_chunk_size=self.kv_chunk_size)
+
+    def _capture(self):
+        # one eager pass per size first: module loading and per-kernel set-up
+        # (shared-memory attributes) happen outside any capture
+        for bs in self.graph_bs:
+            self._step(bs)
+        torch.cuda.synchronize(self.k_cache.device)
+        pool = None
+        for bs in reversed(self.graph_bs):      # largest first, sharing one pool
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, pool=pool):
+                self._step(bs)
+            if pool is None:
+                pool = g.pool()
+            self.graphs[bs] = g
+
+    def padded_size(self, n):
+        i = bisect.bisect_left(self.graph_bs, n)
+        if i == len(self.graph_bs):
+            raise ValueError(f"batch of {n} exceeds the largest captured size {self.max_bs}")
+        return self.graph_bs[i]
+
+    def load(self, q, new_k, new_v, slot_mapping, block_tables, context_lens):
+        """Copy one step's inputs into the static buffers (padding the rest); returns the padded size."""
+        n = q.shape[0]
+        bs = self.padded_size(n)
+        self.q[:n].copy_(q, non_blocking=True)
+        self.new_k[:n].copy_(new_k, non_blocking=True)
+        self.new_v[:n].copy_(new_v, non_blocking=True)
+        self.slot_mapping[:n].copy_(slot_mapping, non_blocking=True)
+        self.slot_mapping[n:bs].fill_(-1)
+        w = block_tables.shape[1]
+        if w > self.max_blocks_per_seq:
+            raise ValueError("block tables are wider than the captured width")
+        self.block_tables[:n, :w].copy_(block_tables, non_blocking=True)
+        self.block_tables[:n, w:].fill_(-1)
+        self.context_lens[:n].copy_(context_lens, non_blocking=True)
+        self.context_lens[n:bs].fill_(0)
+        return bs
+
+    def replay(self, bs):
+        self.graphs[bs].replay()
+
+    def run(self, q, new_k, new_v, slot_mapping, block_tables, context_lens):
+        """Store the new rows and decode one step for a batch of q.shape[0] sequences; returns out[:n]."""
+        bs = self.load(q, new_k, new_v, slot_mapping, block_tables, context_lens)
+        self.replay(bs)
+        return self.out[:q.shape[0]]

@@ -1,0 +1,45 @@
+"""CUDA-graph capture of the store + decode step (captured at the batch sizes
+of "Architektur im Überblick", CUDA Graph Optimierung), against eager calls
+and the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_331_b200 as pa
+from paged_kv_cache_331_b200 import workloads as W
+from paged_kv_cache_331_b200.graphs import DecodeGraphRunner, graph_batch_sizes
+from gpu_helpers import DeviceDecode, assert_attention_close, host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def test_graph_batch_sizes_follow_the_engine():
+    assert graph_batch_sizes(64) == [1, 2, 4, 8, 16, 32, 48, 64]
+    assert graph_batch_sizes(20) == [1, 2, 4, 8, 16]
+
+
+@pytest.mark.parametrize("n", [20, 1, 5, 16, 32])
+def test_graph_replay_matches_eager_and_oracle(oracle, n):
+    rng = np.random.default_rng(100 + n)
+    lens = rng.integers(1, 1500, size=n).astype(np.int32)
+    w = W.decode_workload(lens, 8, 2, 128, 256, rng=rng)
+    dw = DeviceDecode(w)
+    chunk = 256
+    runner = DecodeGraphRunner(dw.k_cache, dw.v_cache, w.num_heads, max_bs=32, max_blocks_per_seq=8,
+                               max_context_len=2048, scale=w.scale, kv_chunk_size=chunk)
+    # the graph path stores the new rows itself; the eager reference works on its own copy of the cache
+    kc2, vc2 = dw.k_cache.clone(), dw.v_cache.clone()
+    out_g = runner.run(dw.q, dw.new_k, dw.new_v, dw.slot_mapping, dw.block_tables, dw.context_lens).clone()
+    pa.store_kvcache(dw.new_k, dw.new_v, kc2, vc2, dw.slot_mapping)
+    out_e = pa.decode(dw.q, kc2, vc2, dw.block_tables, dw.context_lens, 2048, w.scale, kv_chunk_size=chunk)
+    torch.cuda.synchronize()
+    assert torch.equal(dw.k_cache.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(out_g.view(torch.int16), out_e.view(torch.int16))
+    oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
+    _, ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
+    assert_attention_close(out_g, ref, what=f"graph replay n={n}")
+    # a second replay of the same step is bitwise identical
+    out_g2 = runner.run(dw.q, dw.new_k, dw.new_v, dw.slot_mapping, dw.block_tables, dw.context_lens)
+    torch.cuda.synchronize()
+    assert torch.equal(out_g.view(torch.int16), out_g2.view(torch.int16))
+    assert pa.device_error() == 0
