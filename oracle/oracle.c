@@ -30,9 +30,11 @@
  *  - "Architektur im Überblick", "Attention-Mechanismus": GQA through a
  *    separate num_kv_heads; query head h reads kv head h / (num_heads /
  *    num_kv_heads).
+ *  - "Nano-vLLM 源碼學習", layers, 7 (rotary_embedding.py): rotary position
+ *    embedding of q and k from sines and cosines of the position.
  *
  * Every function validates its arguments and returns 0 on success or a
- * negative code: -1 bad argument, -2 block id or slot out of range.
+ * negative code: -1 bad argument, -2 block id, slot or position out of range.
  */
 #include <math.h>
 #include <stdint.h>
@@ -428,6 +430,125 @@ int oracle_prefill_varlen(uint16_t* out, double* out_f64, const uint16_t* q, con
         free(o);
     }
     return err;
+}
+
+/* ----------------------------------------------------------------- rope --- */
+
+/* Rotary position embedding.  "Nano-vLLM 源碼學習", layers, 7 (rotary_embedding.py):
+ * the RotaryEmbedding class adds position information to the query and the key
+ * through sines and cosines of the position; "Architektur im Überblick",
+ * Attention-Mechanismus: the attention layer applies its rotary_emb to q and k
+ * before attention.  The pages print no formula.  Read as RoFormer's rotation
+ * over the whole head, element i paired with element i + D/2 (the layout of
+ * the Qwen models the pages serve), for frequency index i in [0, D/2):
+ *
+ *   theta_i   = base^(-2i/D)
+ *   y_i       = x_i cos(p theta_i) - x_{i+D/2} sin(p theta_i)
+ *   y_{i+D/2} = x_{i+D/2} cos(p theta_i) + x_i sin(p theta_i)
+ *
+ * i.e. the complex number x_i + j x_{i+D/2} multiplied by e^{j p theta_i}. */
+
+static double rope_theta(int32_t i, int32_t head_dim, double base)
+{
+#if ORACLE_MUTANT == 13
+    return pow(base, -(double)i / head_dim);                   /* exponent halved */
+#else
+    return pow(base, -2.0 * i / head_dim);
+#endif
+}
+
+/* The cos/sin cache: row p holds cos(p theta_i) for i in [0, D/2) followed by
+ * sin(p theta_i), each computed in double and rounded once to float. */
+int oracle_rope_table(float* table, int32_t max_position, int32_t head_dim, double base)
+{
+    if (!table || max_position <= 0 || head_dim <= 0 || head_dim % 2 || !(base > 1.0)) return -1;
+    const int32_t half = head_dim / 2;
+    for (int32_t p = 0; p < max_position; ++p)
+        for (int32_t i = 0; i < half; ++i) {
+            double a = (double)p * rope_theta(i, head_dim, base);
+            table[(int64_t)p * head_dim + i] = (float)cos(a);
+#if ORACLE_MUTANT == 12
+            table[(int64_t)p * head_dim + half + i] = (float)-sin(a);   /* rotation by -angle */
+#else
+            table[(int64_t)p * head_dim + half + i] = (float)sin(a);
+#endif
+        }
+    return 0;
+}
+
+/* Rotate one head row x (head_dim bf16) to position row cs of the table;
+ * the products and sums in double, each output rounded once to bf16. */
+static void rope_row(uint16_t* y, double* y64, const uint16_t* x, const float* cs, int32_t head_dim)
+{
+    const int32_t half = head_dim / 2;
+    for (int32_t i = 0; i < half; ++i) {
+#if ORACLE_MUTANT == 11
+        int32_t lo = 2 * i, hi = 2 * i + 1;                    /* adjacent pairs */
+#else
+        int32_t lo = i, hi = i + half;
+#endif
+        double c = cs[i], s = cs[half + i];
+        double a = bf16_to_double(x[lo]), b = bf16_to_double(x[hi]);
+        double ylo = a * c - b * s, yhi = b * c + a * s;
+        y[lo] = double_to_bf16(ylo);
+        y[hi] = double_to_bf16(yhi);
+        if (y64) { y64[lo] = ylo; y64[hi] = yhi; }
+    }
+}
+
+/* Rotary embedding fused with store_kvcache: for every token t at position
+ * positions[t], rotate its num_heads query rows into q_out ([num_tokens,
+ * num_heads, head_dim], dense) and its num_kv_heads key rows; then, if
+ * slot_mapping[t] != -1, store the rotated key rows and the unchanged value
+ * rows exactly as oracle_store_kvcache does. */
+int oracle_rope_store_kvcache(uint16_t* q_out, double* q_out_f64, const uint16_t* q, int64_t q_row_stride,
+                              const uint16_t* key, const uint16_t* value, int64_t key_row_stride,
+                              int64_t value_row_stride, const int32_t* positions, const float* table,
+                              int32_t max_position, uint16_t* k_cache, uint16_t* v_cache,
+                              const int32_t* slot_mapping, int32_t num_tokens, int32_t num_heads,
+                              int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks)
+{
+    if (num_tokens < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 2 || block_size <= 0 ||
+        num_blocks < 0 || max_position <= 0)
+        return -1;
+    if (num_tokens == 0) return 0;
+    if (!q_out || !q || !key || !value || !positions || !table || !k_cache || !v_cache || !slot_mapping) return -1;
+    const int64_t qrow = (int64_t)num_heads * head_dim, kvrow = (int64_t)num_kv_heads * head_dim;
+    if (q_row_stride < qrow || key_row_stride < kvrow || value_row_stride < kvrow) return -1;
+    for (int32_t t = 0; t < num_tokens; ++t) {
+        int32_t p = positions[t];
+        if (p < 0 || p >= max_position) return -2;
+    }
+    uint16_t* krot = (uint16_t*)malloc((size_t)kvrow * sizeof(uint16_t));
+    if (!krot) return -1;
+    for (int32_t t = 0; t < num_tokens; ++t) {
+#if ORACLE_MUTANT == 15
+        const float* cs = table + (int64_t)(positions[t] + 1 < max_position ? positions[t] + 1 : positions[t]) * head_dim;
+#else
+        const float* cs = table + (int64_t)positions[t] * head_dim;
+#endif
+        for (int32_t h = 0; h < num_heads; ++h) {
+            int64_t o = ((int64_t)t * num_heads + h) * head_dim;
+            rope_row(q_out + o, q_out_f64 ? q_out_f64 + o : NULL, q + (int64_t)t * q_row_stride + (int64_t)h * head_dim,
+                     cs, head_dim);
+        }
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            const uint16_t* kx = key + (int64_t)t * key_row_stride + (int64_t)h * head_dim;
+#if ORACLE_MUTANT == 14
+            memcpy(krot + (int64_t)h * head_dim, kx, (size_t)head_dim * sizeof(uint16_t));   /* key not rotated */
+#else
+            rope_row(krot + (int64_t)h * head_dim, NULL, kx, cs, head_dim);
+#endif
+        }
+        int rc = oracle_store_kvcache(krot, value + (int64_t)t * value_row_stride, kvrow, value_row_stride, k_cache,
+                                      v_cache, slot_mapping + t, 1, num_kv_heads, head_dim, block_size, num_blocks);
+        if (rc) {
+            free(krot);
+            return rc;
+        }
+    }
+    free(krot);
+    return 0;
 }
 
 int oracle_mutant_id(void) { return ORACLE_MUTANT; }

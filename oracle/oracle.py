@@ -22,6 +22,7 @@ _c_i32p = ctypes.POINTER(ctypes.c_int32)
 _c_u16p = ctypes.POINTER(ctypes.c_uint16)
 _c_f64p = ctypes.POINTER(ctypes.c_double)
 _c_u8p = ctypes.POINTER(ctypes.c_uint8)
+_c_f32p = ctypes.POINTER(ctypes.c_float)
 
 
 def library_path(mutant: int = 0) -> Path:
@@ -59,9 +60,12 @@ class Oracle:
         L.oracle_merge_partials.argtypes = [_c_u16p, _c_f64p, _c_f64p, _c_f64p, _c_f64p, i32, i32, i32]
         L.oracle_prefill_varlen.argtypes = [_c_u16p, _c_f64p, _c_u16p, _c_u16p, _c_u16p, _c_i32p, _c_i32p,
                                             _c_i32p, i32, i32, i32, i32, i32, i32, i32, f64, i32, _c_u8p, ci]
+        L.oracle_rope_table.argtypes = [_c_f32p, i32, i32, f64]
+        L.oracle_rope_store_kvcache.argtypes = [_c_u16p, _c_f64p, _c_u16p, i64, _c_u16p, _c_u16p, i64, i64, _c_i32p,
+                                                _c_f32p, i32, _c_u16p, _c_u16p, _c_i32p, i32, i32, i32, i32, i32, i32]
         for name in ("oracle_bf16_round", "oracle_kv_location", "oracle_store_kvcache", "oracle_decode",
                      "oracle_decode_partials", "oracle_merge_partials", "oracle_prefill_varlen",
-                     "oracle_mutant_id", "oracle_max_threads"):
+                     "oracle_rope_table", "oracle_rope_store_kvcache", "oracle_mutant_id", "oracle_max_threads"):
             getattr(L, name).restype = ctypes.c_int
         assert L.oracle_mutant_id() == mutant
 
@@ -106,6 +110,37 @@ class Oracle:
         self._check(self.lib.oracle_store_kvcache(self._p(key2, _c_u16p), self._p(val2, _c_u16p), ks, vs,
                                                   self._p(k_cache, _c_u16p), self._p(v_cache, _c_u16p),
                                                   self._p(sm, _c_i32p), n, hkv, d, bs, nb), "store_kvcache")
+
+    def rope_table(self, max_position, head_dim, base):
+        """Rotary cos/sin cache [max_position, head_dim] float32: cos(p theta_i) then sin(p theta_i)."""
+        t = np.empty((max_position, head_dim), dtype=np.float32)
+        self._check(self.lib.oracle_rope_table(self._p(t, _c_f32p), max_position, head_dim, float(base)), "rope_table")
+        return t
+
+    def rope_store_kvcache(self, q, key, value, positions, table, k_cache, v_cache, slot_mapping, *, want_f64=False):
+        """Rotate q ([N, Hq, D], row stride may exceed Hq*D) and key to their positions; store the rotated key
+        and the value rows into the cache (slot -1 skipped).  Returns q_out [N, Hq, D] (and its doubles)."""
+        assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+        nb, bs, hkv, d = k_cache.shape
+        n = int(np.asarray(positions).shape[0])
+        hq = q.shape[1]
+        pos = np.ascontiguousarray(positions, dtype=np.int32)
+        sm = np.ascontiguousarray(slot_mapping, dtype=np.int32)
+        tab = np.ascontiguousarray(table, dtype=np.float32)
+        rows = []
+        for a, h in ((q, hq), (key, hkv), (value, hkv)):
+            a2 = a.reshape(n, -1) if n else np.zeros((0, h * d), np.uint16)
+            assert a2.strides[-1] == 2
+            rows.append((a2, a2.strides[0] // 2 if n else h * d))
+        out = np.zeros((n, hq, d), dtype=np.uint16)
+        of = np.zeros((n, hq, d), dtype=np.float64) if want_f64 else None
+        (q2, qs), (k2, ks), (v2, vs) = rows
+        self._check(self.lib.oracle_rope_store_kvcache(
+            self._p(out, _c_u16p), self._p(of, _c_f64p), self._p(q2, _c_u16p), qs, self._p(k2, _c_u16p),
+            self._p(v2, _c_u16p), ks, vs, self._p(pos, _c_i32p), self._p(tab, _c_f32p), tab.shape[0],
+            self._p(k_cache, _c_u16p), self._p(v_cache, _c_u16p), self._p(sm, _c_i32p), n, hq, hkv, d, bs, nb),
+            "rope_store_kvcache")
+        return (out, of) if want_f64 else out
 
     def decode(self, q, k_cache, v_cache, block_tables, context_lens, scale, *, want_f64=False, nthreads=0):
         q = np.ascontiguousarray(q, dtype=np.uint16)
