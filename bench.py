@@ -355,6 +355,7 @@ def bench_prefill(args, dev, peaks):
     tflops = flops / (prefill_ms / 1e3) / 1e12
     store_bytes = 2 * 2 * int(w.cu_seqlens_q[-1]) * w.num_kv_heads * w.head_dim * 2 + 4 * int(w.cu_seqlens_q[-1])
     store_gbs = store_bytes / (store_ms / 1e3) / 1e9
+    rot = bench_rotary_store(w, dev, q, nk, nv, kc, vc, slots, flush, reps)
     peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     return {
         "workload": w.name, "num_seqs": w.num_seqs, "prefix_len": 1024, "suffix": "U[64,512]",
@@ -364,8 +365,45 @@ def bench_prefill(args, dev, peaks):
                      "peak_kind": f"bf16 burst ({peaks.get('source')})"},
         "store": {"rows": int(w.cu_seqlens_q[-1]), "ms": store_ms, "gbs": store_gbs,
                   "frac": store_gbs / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "bytes": store_bytes},
+        "rotary_store": rot,
         "gpu_launches_per_rep": 2,
     }
+
+
+def bench_rotary_store(w, dev, q, nk, nv, kc, vc, slots, flush, reps):
+    """The prefill's new tokens through the fused rotary + store kernel (q rotated into a new buffer, rotated keys
+    and values into the cache), L2 flushed between reps."""
+    import torch
+    import paged_kv_cache_331_b200 as pa
+    n = int(w.cu_seqlens_q[-1])
+    lq = np.diff(w.cu_seqlens_q)
+    cached = np.diff(w.cu_seqlens_k) - lq
+    pos_h = np.concatenate([c + np.arange(l) for c, l in zip(cached, lq)]).astype(np.int32)
+    max_pos = 40960
+    table = pa.rotary_cos_sin_cache(max_pos, w.head_dim, 1e6, device=dev)
+    pos = to_dev(pos_h, "i32", dev)
+    q_rot = torch.empty_like(q)
+    for _ in range(3):
+        pa.rotary_store_kvcache(q, nk, nv, pos, table, kc, vc, slots, out=q_rot)
+    torch.cuda.synchronize(dev)
+    ev = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(); pa.rotary_store_kvcache(q, nk, nv, pos, table, kc, vc, slots, out=q_rot); b.record()
+        ev.append((a, b))
+    torch.cuda.synchronize(dev)
+    assert pa.device_error() == 0
+    ms = float(np.median([x.elapsed_time(y) for x, y in ev]))
+    qb = n * w.num_heads * w.head_dim * 2
+    kvb = n * w.num_kv_heads * w.head_dim * 2
+    live = int((w.slot_mapping >= 0).sum())
+    lkvb = live * w.num_kv_heads * w.head_dim * 2
+    alg = (qb + 2 * kvb + 8 * n + len(np.unique(pos_h)) * w.head_dim * 4) + (qb + 2 * lkvb)
+    gbs = alg / (ms / 1e3) / 1e9
+    return {"tokens": n, "ms": ms, "bytes": alg, "gbs": gbs, "frac": gbs / load_peaks().get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+            "bytes_rule": "read q, k, v rows, positions, slots and each distinct table row once; write rotated q "
+                          "and the stored k/v rows"}
 
 
 def bench_graph(args, dev):

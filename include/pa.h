@@ -5,6 +5,8 @@
  * engine over a paged KV cache:
  *
  *   pa_store_kvcache   scatter the new tokens' K/V rows into cache slots
+ *   pa_rotary_store_kvcache
+ *                      rotary embedding of q and k fused with that scatter
  *   pa_decode          one query token per sequence against its cached keys
  *                      (GQA; long contexts split across CTAs + a merge pass)
  *   pa_prefill_varlen  causal varlen prefill whose leading blocks may be
@@ -13,7 +15,8 @@
  * Conventions shared by every entry point
  * ----------------------------------------
  * - Pointers named *_cache, q, out, key, value, block_tables, context_lens,
- *   cu_seqlens_*, slot_mapping and workspace are DEVICE pointers owned by the
+ *   cu_seqlens_*, slot_mapping, positions, cos_sin_cache, table and workspace
+ *   are DEVICE pointers owned by the
  *   caller.  The library never allocates, frees or retains them.
  * - bf16 tensors are passed as void*; their layouts are stated per argument.
  *   Every tensor is dense row-major unless a row stride is given.
@@ -94,6 +97,57 @@ PA_API pa_status pa_store_kvcache(const void* key, const void* value, int64_t ke
                            void* k_cache, void* v_cache, const int32_t* slot_mapping, int32_t num_tokens,
                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
                            void* stream);
+
+/*
+ * pa_rotary_cos_sin_cache -- fill the rotary embedding's cos/sin table.
+ * ("Nano-vLLM 源碼學習", layers, 7 rotary_embedding.py: the RotaryEmbedding
+ * class encodes positions through sines and cosines, built once and cached.)
+ *
+ * For p in [0, max_position) and i in [0, head_dim/2), with
+ * theta_i = base^(-2i/head_dim) and the angle p*theta_i taken in double:
+ *   table[p*head_dim + i]              = (float) cos(p*theta_i)
+ *   table[p*head_dim + head_dim/2 + i] = (float) sin(p*theta_i)
+ * table: caller-owned device buffer of max_position*head_dim floats.
+ * head_dim even in [2, 1024]; base > 1; max_position*head_dim < 2^31.
+ */
+PA_API pa_status pa_rotary_cos_sin_cache(float* table, int32_t max_position, int32_t head_dim, double base,
+                                  void* stream);
+
+/*
+ * pa_rotary_store_kvcache -- rotary position embedding of q and k fused with
+ * pa_store_kvcache.  ("Nano-vLLM 源碼學習", layers, 7 rotary_embedding.py and
+ * §二.2; "Architektur im Überblick", Attention-Mechanismus: rotary_emb is
+ * applied to q and k before attention stores k and v in the cache.)
+ *
+ * For every token t at position p = positions[t], each head row x (head_dim
+ * values) of q[t] and key[t] is rotated pairwise, element i with element
+ * i + head_dim/2, by the angle whose cos/sin sit in row p of cos_sin_cache:
+ *   y_i = x_i cos - x_{i+D/2} sin,   y_{i+D/2} = x_{i+D/2} cos + x_i sin
+ * in float, rounded to bf16 (nearest-even).  The rotated query rows go to
+ * q_out; if s = slot_mapping[t] != -1 the rotated key rows and the unchanged
+ * value rows are written to slot s exactly as pa_store_kvcache writes them.
+ *
+ * q:             [num_tokens, num_heads, head_dim] bf16, row t at element
+ *                t*q_row_stride (views into a fused QKV buffer allowed).
+ * q_out:         [num_tokens, num_heads, head_dim] bf16, dense.  May be q
+ *                itself when q_row_stride == num_heads*head_dim; must not
+ *                otherwise overlap q, key or value.
+ * key, value:    as for pa_store_kvcache.
+ * positions:     [num_tokens] int32 in [0, max_position).  A position
+ *                outside that range leaves the token's q_out rows and K cache
+ *                rows unwritten and sets device error code 4.
+ * cos_sin_cache: [max_position, head_dim] float as pa_rotary_cos_sin_cache
+ *                fills it.
+ * Requires head_dim 64 or 128, every pointer 16-byte aligned and every row
+ * stride a multiple of 8 elements (PA_ERR_UNSUPPORTED otherwise).
+ * num_tokens == 0 launches nothing and returns PA_OK.
+ */
+PA_API pa_status pa_rotary_store_kvcache(void* q_out, const void* q, int64_t q_row_stride, const void* key,
+                                  const void* value, int64_t key_row_stride, int64_t value_row_stride,
+                                  const int32_t* positions, const float* cos_sin_cache, int32_t max_position,
+                                  void* k_cache, void* v_cache, const int32_t* slot_mapping, int32_t num_tokens,
+                                  int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                  int32_t num_blocks, void* stream);
 
 /*
  * pa_decode_chunk_size -- tokens per split-KV chunk that pa_decode uses when
@@ -207,8 +261,11 @@ PA_API pa_status pa_prefill_varlen(void* out, const void* q, const void* k_cache
 /*
  * pa_device_error -- read and clear the library's device-side error word on
  * the current device (synchronises the given stream).  Kernels set it instead
- * of hanging when a pipeline wait exceeds its time limit (about one second);
- * 0 means no error.  Diagnostic only.
+ * of hanging when a pipeline wait exceeds its time limit (about one second),
+ * and pa_rotary_store_kvcache sets it for a position outside its table.
+ * Codes: 0 none, 1 a pipeline wait timed out, 2 the wait for in-flight copies
+ * at exit timed out, 3 dynamic shared memory misaligned, 4 rotary position
+ * out of range.  Diagnostic only.
  */
 PA_API pa_status pa_device_error(int32_t* code_out, void* stream);
 

@@ -31,6 +31,9 @@ _PROTOS = {
     "pa_prefill_varlen": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _i32, _i32, _i32,
                                          _i32, _i32, _i32, _f32, _i32, _vp]),
     "pa_device_error": (ctypes.c_int, [ctypes.POINTER(_i32), _vp]),
+    "pa_rotary_cos_sin_cache": (ctypes.c_int, [_vp, _i32, _i32, ctypes.c_double, _vp]),
+    "pa_rotary_store_kvcache": (ctypes.c_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _vp,
+                                               _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pa_decode_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                          _f32, _i32, _vp]),
 }
@@ -93,6 +96,53 @@ def store_kvcache(key, value, k_cache, v_cache, slot_mapping, stream=None) -> No
         _check(lib().pa_store_kvcache(key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0),
                                       k_cache.data_ptr(), v_cache.data_ptr(), slot_mapping.data_ptr(), n, hkv, d, bs,
                                       nb, _stream(k_cache, stream)), "pa_store_kvcache")
+
+
+def rotary_cos_sin_cache(max_position, head_dim, base, device=None, stream=None) -> torch.Tensor:
+    """pa_rotary_cos_sin_cache: a new [max_position, head_dim] float32 table, cos(p theta_i) | sin(p theta_i)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    table = torch.empty(max_position, head_dim, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().pa_rotary_cos_sin_cache(table.data_ptr(), max_position, head_dim, float(base),
+                                             _stream(table, stream)), "pa_rotary_cos_sin_cache")
+    return table
+
+
+def rotary_store_kvcache(q, key, value, positions, cos_sin_cache, k_cache, v_cache, slot_mapping, *, out=None,
+                         stream=None) -> torch.Tensor:
+    """pa_rotary_store_kvcache: rotate q [N, Hq, D] and key [N, Hkv, D] to their positions, store the rotated key and
+    the value into the cache at slot_mapping (-1 = skip); returns the rotated q ([N, Hq, D], dense; ``out`` may be
+    q itself when q is dense)."""
+    for n, t in (("q", q), ("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _cuda(t, n, torch.bfloat16)
+    _cuda(positions, "positions", torch.int32)
+    _cuda(slot_mapping, "slot_mapping", torch.int32)
+    _cuda(cos_sin_cache, "cos_sin_cache", torch.float32)
+    for n, t in (("k_cache", k_cache), ("v_cache", v_cache), ("positions", positions), ("slot_mapping", slot_mapping),
+                 ("cos_sin_cache", cos_sin_cache)):
+        _dense(t, n)
+    nb, bs, hkv, d = k_cache.shape
+    n, hq = q.shape[0], q.shape[1]
+    if tuple(q.shape[1:]) != (hq, d) or q.stride(-1) != 1 or q.stride(-2) != d:
+        raise ValueError(f"q must be [N, Hq, {d}] with dense rows")
+    for name, t in (("key", key), ("value", value)):
+        if t.shape[0] != n or tuple(t.shape[1:]) != (hkv, d) or t.stride(-1) != 1 or t.stride(-2) != d:
+            raise ValueError(f"{name} must be [N, {hkv}, {d}] with dense rows")
+    if positions.shape != (n,) or slot_mapping.shape != (n,):
+        raise ValueError("positions and slot_mapping must be [N]")
+    if cos_sin_cache.dim() != 2 or cos_sin_cache.shape[1] != d:
+        raise ValueError(f"cos_sin_cache must be [max_position, {d}]")
+    if out is None:
+        out = torch.empty(n, hq, d, dtype=torch.bfloat16, device=q.device)
+    _cuda(out, "out", torch.bfloat16)
+    _dense(out, "out")
+    with torch.cuda.device(k_cache.device):
+        _check(lib().pa_rotary_store_kvcache(out.data_ptr(), q.data_ptr(), q.stride(0), key.data_ptr(),
+                                             value.data_ptr(), key.stride(0), value.stride(0), positions.data_ptr(),
+                                             cos_sin_cache.data_ptr(), cos_sin_cache.shape[0], k_cache.data_ptr(),
+                                             v_cache.data_ptr(), slot_mapping.data_ptr(), n, hq, hkv, d, bs, nb,
+                                             _stream(k_cache, stream)), "pa_rotary_store_kvcache")
+    return out
 
 
 def decode_chunk_size(num_seqs, num_kv_heads, max_context_len, block_size) -> int:

@@ -159,6 +159,88 @@ pa_status pa_store_kvcache(const void* key, const void* value, int64_t key_row_s
   return PA_OK;
 }
 
+pa_status pa_rotary_cos_sin_cache(float* table, int32_t max_position, int32_t head_dim, double base, void* stream) {
+  t_last_error[0] = 0;
+  if (!table) return fail(PA_ERR_INVALID_ARG, "rotary_cos_sin_cache: null table");
+  if (max_position <= 0 || head_dim < 2 || head_dim > 1024 || head_dim % 2)
+    return fail(PA_ERR_INVALID_ARG, "rotary_cos_sin_cache: need max_position > 0 and an even head_dim in [2, 1024]");
+  if (!(base > 1.0)) return fail(PA_ERR_INVALID_ARG, "rotary_cos_sin_cache: base must be > 1");
+  if (static_cast<int64_t>(max_position) * head_dim >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID_ARG, "rotary_cos_sin_cache: max_position*head_dim must be < 2^31");
+  cudaError_t e = launch_rotary_table(table, max_position, head_dim, base, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "rotary_cos_sin_cache launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
+static bool ranges_overlap(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + b_bytes && y < x + a_bytes;
+}
+
+pa_status pa_rotary_store_kvcache(void* q_out, const void* q, int64_t q_row_stride, const void* key,
+                                  const void* value, int64_t key_row_stride, int64_t value_row_stride,
+                                  const int32_t* positions, const float* cos_sin_cache, int32_t max_position,
+                                  void* k_cache, void* v_cache, const int32_t* slot_mapping, int32_t num_tokens,
+                                  int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                  int32_t num_blocks, void* stream) {
+  t_last_error[0] = 0;
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "rotary_store_kvcache: num_tokens < 0");
+  if (num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0 ||
+      max_position <= 0)
+    return fail(PA_ERR_INVALID_ARG,
+                "rotary_store_kvcache: num_heads, num_kv_heads, head_dim, block_size, num_blocks, max_position "
+                "must be > 0");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "rotary_store_kvcache: head_dim %d (supported: 64, 128)", head_dim);
+  if (num_heads > 4096 || num_kv_heads > 4096)
+    return fail(PA_ERR_UNSUPPORTED, "rotary_store_kvcache: more than 4096 heads");
+  const int64_t qrow = static_cast<int64_t>(num_heads) * head_dim;
+  const int64_t kvrow = static_cast<int64_t>(num_kv_heads) * head_dim;
+  if (q_row_stride < qrow || key_row_stride < kvrow || value_row_stride < kvrow)
+    return fail(PA_ERR_INVALID_ARG, "rotary_store_kvcache: row strides shorter than the rows");
+  if (static_cast<int64_t>(max_position) * head_dim >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID_ARG, "rotary_store_kvcache: max_position*head_dim must be < 2^31");
+  if (num_tokens == 0) return PA_OK;
+  if (!q_out || !q || !key || !value || !positions || !cos_sin_cache || !k_cache || !v_cache || !slot_mapping)
+    return fail(PA_ERR_INVALID_ARG, "rotary_store_kvcache: null pointer");
+  auto al16 = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
+  if (!al16(q_out) || !al16(q) || !al16(key) || !al16(value) || !al16(cos_sin_cache) || !al16(k_cache) ||
+      !al16(v_cache) || q_row_stride % 8 || key_row_stride % 8 || value_row_stride % 8)
+    return fail(PA_ERR_UNSUPPORTED,
+                "rotary_store_kvcache: pointers must be 16-byte aligned and row strides multiples of 8 elements");
+  const size_t out_bytes = static_cast<size_t>(num_tokens) * qrow * 2;
+  const bool in_place = q_out == q && q_row_stride == qrow;
+  auto span = [&](int64_t stride, int64_t row) {
+    return (static_cast<size_t>(num_tokens - 1) * stride + row) * 2;
+  };
+  if ((!in_place && ranges_overlap(q_out, out_bytes, q, span(q_row_stride, qrow))) ||
+      ranges_overlap(q_out, out_bytes, key, span(key_row_stride, kvrow)) ||
+      ranges_overlap(q_out, out_bytes, value, span(value_row_stride, kvrow)))
+    return fail(PA_ERR_INVALID_ARG, "rotary_store_kvcache: q_out overlaps q (other than in place), key or value");
+  RotaryArgs a{};
+  a.q_out = q_out;
+  a.q = q;
+  a.key = key;
+  a.value = value;
+  a.positions = positions;
+  a.cos_sin = cos_sin_cache;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.slot_mapping = slot_mapping;
+  a.q_row_stride = q_row_stride;
+  a.key_row_stride = key_row_stride;
+  a.value_row_stride = value_row_stride;
+  a.num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  a.max_position = max_position;
+  a.num_tokens = num_tokens;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  cudaError_t e = launch_rotary_store(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "rotary_store_kvcache launch: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
 int32_t pa_decode_chunk_size(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int32_t block_size) {
   if (num_seqs < 0 || num_kv_heads <= 0 || max_context_len < 0 || block_size <= 0) return -1;
   return decode_auto_chunk(num_seqs, num_kv_heads, max_context_len, current_device_info()->sm_count);

@@ -16,6 +16,7 @@ enum DeviceErrorCode : unsigned int {
   kErrWaitTimeout = 1,     // an mbarrier wait ran out of time
   kErrDrainTimeout = 2,    // waiting for in-flight copies at exit ran out of time
   kErrSmemAlign = 3,       // dynamic shared memory not 1024-byte aligned
+  kErrBadPosition = 4,     // a rotary position outside [0, max_position)
 };
 
 #ifndef PA_WAIT_LIMIT_NS

@@ -36,6 +36,31 @@ cudaError_t launch_store_kvcache(const void* key, const void* value, int64_t key
                                  const int32_t* slot_mapping, int32_t num_tokens, int32_t row_elems,
                                  int64_t num_slots, cudaStream_t stream);
 
+// ----------------------------------------------------------------- rotary --
+struct RotaryArgs {
+  void* q_out;                 // [num_tokens, num_heads, head_dim], dense
+  const void* q;               // row stride q_row_stride (elements)
+  const void* key;             // row stride key_row_stride
+  const void* value;           // row stride value_row_stride
+  const int32_t* positions;    // [num_tokens]
+  const float* cos_sin;        // [max_position, head_dim]: cos | sin
+  void* k_cache;
+  void* v_cache;
+  const int32_t* slot_mapping;
+  int64_t q_row_stride;
+  int64_t key_row_stride;
+  int64_t value_row_stride;
+  int64_t num_slots;
+  int32_t max_position;
+  int32_t num_tokens;
+  int32_t num_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+};
+cudaError_t launch_rotary_store(const RotaryArgs& a, cudaStream_t stream);
+cudaError_t launch_rotary_table(float* table, int32_t max_position, int32_t head_dim, double base,
+                                cudaStream_t stream);
+
 // ----------------------------------------------------------------- decode --
 struct DecodeArgs {
   void* out;

@@ -1,14 +1,17 @@
-"""CUDA-graph capture of the decode step (store_kvcache + decode).
+"""CUDA-graph capture of the decode step ([rotary +] store_kvcache + decode).
 
 "Architektur im Überblick", section "CUDA Graph Optimierung": the engine
 captures its decode step once per batch size in [1, 2, 4, 8] + [16, 32, ...,
 max_bs], in descending order and into one shared memory pool, and replays
 the smallest captured graph that holds the current batch.  This runner does
 the same for the attention step of one layer: the new tokens' K/V rows are
-scattered into the cache and every sequence attends over its blocks.
+scattered into the cache and every sequence attends over its blocks.  Given
+a rotary cos/sin cache, the step first rotates q and the new keys to their
+positions ("Nano-vLLM 源碼學習", layers, 7 rotary_embedding.py), fused with the
+store, and decode reads the rotated q.
 
 Rows past the real batch are padding: their slot is -1 (the store skips them)
-and their context length 0 (decode writes zeros), so a padded replay computes
+their context length 0 (decode writes zeros) and their position 0, so a padded replay computes
 exactly what an unpadded call computes for the real rows.  The KV cache, the
 static input buffers and the decode workspace keep their addresses for the
 runner's lifetime: the captured kernels (and their TMA tensor maps) refer to
@@ -33,7 +36,7 @@ class DecodeGraphRunner:
     """Captured store_kvcache + decode steps for one layer's paged KV cache."""
 
     def __init__(self, k_cache, v_cache, num_heads, max_bs, max_blocks_per_seq, max_context_len, scale,
-                 kv_chunk_size=0):
+                 kv_chunk_size=0, cos_sin_cache=None):
         if not (k_cache.is_cuda and v_cache.is_cuda):
             raise TypeError("the KV cache must live on a CUDA device")
         self.k_cache, self.v_cache = k_cache, v_cache
@@ -50,6 +53,9 @@ class DecodeGraphRunner:
         self.block_tables = torch.full((max_bs, max_blocks_per_seq), -1, dtype=torch.int32, device=dev)
         self.context_lens = torch.zeros(max_bs, dtype=torch.int32, device=dev)
         self.out = torch.zeros(max_bs, num_heads, d, dtype=bf, device=dev)
+        self.cos_sin_cache = cos_sin_cache
+        self.positions = torch.zeros(max_bs, dtype=torch.int32, device=dev)
+        self.q_rot = torch.zeros_like(self.q) if cos_sin_cache is not None else None
         self.graph_bs = graph_batch_sizes(max_bs)
         ws = max(pa.decode_workspace_size(b, num_heads, hkv, d, max_context_len, bs_blk, kv_chunk_size)
                  for b in self.graph_bs)
@@ -58,8 +64,14 @@ class DecodeGraphRunner:
         self._capture()
 
     def _step(self, bs):
-        pa.store_kvcache(self.new_k[:bs], self.new_v[:bs], self.k_cache, self.v_cache, self.slot_mapping[:bs])
-        pa.decode(self.q[:bs], self.k_cache, self.v_cache, self.block_tables[:bs], self.context_lens[:bs],
+        if self.cos_sin_cache is None:
+            pa.store_kvcache(self.new_k[:bs], self.new_v[:bs], self.k_cache, self.v_cache, self.slot_mapping[:bs])
+            q = self.q[:bs]
+        else:
+            q = pa.rotary_store_kvcache(self.q[:bs], self.new_k[:bs], self.new_v[:bs], self.positions[:bs],
+                                        self.cos_sin_cache, self.k_cache, self.v_cache, self.slot_mapping[:bs],
+                                        out=self.q_rot[:bs])
+        pa.decode(q, self.k_cache, self.v_cache, self.block_tables[:bs], self.context_lens[:bs],
                   self.max_context_len, self.scale, out=self.out[:bs], workspace=self.workspace,
                   kv_chunk_size=self.kv_chunk_size)
 
@@ -84,8 +96,9 @@ class DecodeGraphRunner:
             raise ValueError(f"batch of {n} exceeds the largest captured size {self.max_bs}")
         return self.graph_bs[i]
 
-    def load(self, q, new_k, new_v, slot_mapping, block_tables, context_lens):
-        """Copy one step's inputs into the static buffers (padding the rest); returns the padded size."""
+    def load(self, q, new_k, new_v, slot_mapping, block_tables, context_lens, positions=None):
+        """Copy one step's inputs into the static buffers (padding the rest); returns the padded size.
+        ``positions`` (the new tokens' positions) is required when the runner rotates."""
         n = q.shape[0]
         bs = self.padded_size(n)
         self.q[:n].copy_(q, non_blocking=True)
@@ -100,13 +113,18 @@ class DecodeGraphRunner:
         self.block_tables[:n, w:].fill_(-1)
         self.context_lens[:n].copy_(context_lens, non_blocking=True)
         self.context_lens[n:bs].fill_(0)
+        if self.cos_sin_cache is not None:
+            if positions is None:
+                raise ValueError("a rotary runner needs the new tokens' positions")
+            self.positions[:n].copy_(positions, non_blocking=True)
+            self.positions[n:bs].fill_(0)
         return bs
 
     def replay(self, bs):
         self.graphs[bs].replay()
 
-    def run(self, q, new_k, new_v, slot_mapping, block_tables, context_lens):
+    def run(self, q, new_k, new_v, slot_mapping, block_tables, context_lens, positions=None):
         """Store the new rows and decode one step for a batch of q.shape[0] sequences; returns out[:n]."""
-        bs = self.load(q, new_k, new_v, slot_mapping, block_tables, context_lens)
+        bs = self.load(q, new_k, new_v, slot_mapping, block_tables, context_lens, positions)
         self.replay(bs)
         return self.out[:q.shape[0]]

@@ -8,7 +8,7 @@ import torch
 import paged_kv_cache_331_b200 as pa
 from paged_kv_cache_331_b200 import workloads as W
 from paged_kv_cache_331_b200.graphs import DecodeGraphRunner, graph_batch_sizes
-from gpu_helpers import DeviceDecode, assert_attention_close, host_bits
+from gpu_helpers import DeviceDecode, assert_attention_close
 
 pytestmark = pytest.mark.gpu
 
@@ -42,4 +42,28 @@ def test_graph_replay_matches_eager_and_oracle(oracle, n):
     out_g2 = runner.run(dw.q, dw.new_k, dw.new_v, dw.slot_mapping, dw.block_tables, dw.context_lens)
     torch.cuda.synchronize()
     assert torch.equal(out_g.view(torch.int16), out_g2.view(torch.int16))
+    assert pa.device_error() == 0
+
+
+@pytest.mark.parametrize("n", [3, 16])
+def test_rotary_graph_replay_matches_eager_and_oracle(oracle, n):
+    rng = np.random.default_rng(200 + n)
+    lens = rng.integers(1, 2000, size=n).astype(np.int32)
+    w = W.decode_workload(lens, 16, 8, 128, 256, rng=rng)
+    dw = DeviceDecode(w)
+    table = oracle.rope_table(2048, 128, 1e6)
+    dtab = torch.from_numpy(table).cuda()
+    pos = torch.from_numpy(lens - 1).cuda()
+    runner = DecodeGraphRunner(dw.k_cache, dw.v_cache, w.num_heads, max_bs=16, max_blocks_per_seq=8,
+                               max_context_len=2048, scale=w.scale, cos_sin_cache=dtab)
+    kc2, vc2 = dw.k_cache.clone(), dw.v_cache.clone()
+    out_g = runner.run(dw.q, dw.new_k, dw.new_v, dw.slot_mapping, dw.block_tables, dw.context_lens, pos).clone()
+    qr = pa.rotary_store_kvcache(dw.q, dw.new_k, dw.new_v, pos, dtab, kc2, vc2, dw.slot_mapping)
+    out_e = pa.decode(qr, kc2, vc2, dw.block_tables, dw.context_lens, 2048, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(dw.k_cache.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(out_g.view(torch.int16), out_e.view(torch.int16))
+    q_rot = oracle.rope_store_kvcache(w.q, w.new_k, w.new_v, lens - 1, table, w.k_cache, w.v_cache, w.slot_mapping)
+    _, ref = oracle.decode(q_rot, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
+    assert_attention_close(out_g, ref, what=f"rotary graph replay n={n}")
     assert pa.device_error() == 0
