@@ -7,9 +7,10 @@
 // start at num_cached_tokens, so query i of a sequence with Lk keys and Lq
 // new tokens sits at position Lk - Lq + i.)
 //
-// Persistent: one CTA per SM walks a static list of work items; a work item
-// is two query tiles (A and B) of one (kv head g, sequence b).  The M = 128 rows of a tile pack the G query heads that share kv head
-// g, QP = 128 / G query positions each (row r -> head g*G + r / QP,
+// Persistent: one CTA per SM takes work items from a device counter until
+// none are left; a work item is two query tiles (A and B) of one (kv head g,
+// sequence b).  The M = 128 rows of a tile pack the G query heads that share
+// kv head g, QP = 128 / G query positions each (row r -> head g*G + r / QP,
 // position qt*QP + r % QP), so every K/V tile loaded serves 2*G heads-tiles.
 // Keys stream in tiles of 128 tokens gathered through the block table (TMA
 // boxes whose row coordinate is block_id * block_size + offset).
@@ -21,8 +22,9 @@
 //              exponentials on the FMA pipe), writes P as bf16 pairs over the
 //              first half of its own S columns, rescales its O row in TMEM when
 //              the running max grows, and does the epilogue.
-//   warp 8     TMA producer: both Q tiles once, then K and V tiles in rings
-//              (K one tile ahead).
+//   warp 8     TMA producer: takes the next item, publishes it to the other
+//              warps through a shared-memory queue, loads its two Q tiles,
+//              then its K and V tiles in rings (K one tile ahead).
 //   warps 10-11 idle (they complete the third warpgroup, whose registers
 //              the softmax warpgroups borrow through setmaxnreg).
 //   warp 9     TMEM allocator and single-thread MMA issuer, in the order
@@ -169,8 +171,8 @@ constexpr float kRescaleLog2 = 8.0f;
 
 // One work item: a pair of query tiles (A = the later one, B) of one
 // (kv head, sequence).  Items are numbered pair-rank-major (rank 0 = the last
-// pair of each sequence, which sees the most keys), so consecutive items have
-// similar cost; each persistent CTA takes every gridDim.x-th item.
+// pair of each sequence, which sees the most keys), so the costliest items
+// are handed out first and items of similar cost run side by side.
 struct Item {
   int b, g;
   int Lq, Lk, q_row0, pos_off;
