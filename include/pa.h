@@ -61,7 +61,8 @@ typedef enum pa_status {
     PA_ERR_INVALID_ARG = 1,
     PA_ERR_UNSUPPORTED = 2,
     PA_ERR_CUDA = 3,
-    PA_ERR_WORKSPACE = 4
+    PA_ERR_WORKSPACE = 4,
+    PA_ERR_NO_FREE_BLOCK = 5   /* block manager (pa_block_manager.h): no free cache block left */
 } pa_status;
 
 /* Static string naming a status code. */

@@ -44,23 +44,29 @@ def _stale(target: Path, inputs) -> bool:
     return any(p.stat().st_mtime > t for p in inputs)
 
 
+CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-fvisibility=hidden", "-Wall", "-Wextra"]
+
+
 def build(force: bool = False, verbose: bool = False) -> Path:
     BUILD.mkdir(exist_ok=True)
-    srcs = sorted(CSRC.glob("*.cu"))
     deps = _deps()
     objs = []
     jobs = []
-    for s in srcs:
+    for s in sorted(CSRC.glob("*.cu")):           # device code and the C ABI
         o = BUILD / (s.stem + ".o")
         objs.append(o)
         if force or _stale(o, [s] + deps):
-            cmd = [nvcc(), *ARCH, *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", "-c", str(s), "-o", str(o)]
-            jobs.append(cmd)
+            jobs.append([nvcc(), *ARCH, *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", "-c", str(s), "-o", str(o)])
+    for s in sorted(CSRC.glob("*.cpp")):          # host-only code (block manager)
+        o = BUILD / (s.stem + "_host.o")
+        objs.append(o)
+        if force or _stale(o, [s] + deps):
+            jobs.append(["g++", *CXX_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", "-c", str(s), "-o", str(o)])
 
     def run(cmd):
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
-            raise RuntimeError(f"nvcc failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
+            raise RuntimeError(f"compile failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
         return r.stdout + r.stderr
 
     if jobs:

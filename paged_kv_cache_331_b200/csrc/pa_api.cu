@@ -127,6 +127,7 @@ const char* pa_status_string(int status) {
     case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
     case PA_ERR_CUDA: return "PA_ERR_CUDA";
     case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+    case PA_ERR_NO_FREE_BLOCK: return "PA_ERR_NO_FREE_BLOCK";
     default: return "PA_ERR_UNKNOWN";
   }
 }
