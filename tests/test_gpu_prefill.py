@@ -37,7 +37,7 @@ CASES = [
     (512, [300, 64], 16, 2, 128, 64, True),
     (32, [9, 20], 4, 4, 64, 16, False),
     (256, [100, 257], 8, 2, 128, 256, False),
-    (300, [100, 40], 8, 2, 128, 512, True),
+    (512, [100, 40], 8, 2, 128, 512, True),
     (0, [700, 3], 4, 4, 64, 1024, True),
 ]
 
