@@ -9,6 +9,9 @@
  *                      rotary embedding of q and k fused with that scatter
  *   pa_decode          one query token per sequence against its cached keys
  *                      (GQA; long contexts split across CTAs + a merge pass)
+ *   pa_decode_partial, pa_merge_partials
+ *                      the same split across GPUs: per-device partials,
+ *                      combined after an all-gather
  *   pa_prefill_varlen  causal varlen prefill whose leading blocks may be
  *                      shared prefix-cache blocks
  *
@@ -229,6 +232,42 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache
                                    const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs,
                                    int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                    int32_t num_blocks, float scale, int32_t kv_chunk_size, void* stream);
+
+/*
+ * pa_decode_partial -- pa_decode over the keys this caller holds, returning
+ * an fp32 partial instead of the bf16 output, so that partials computed on
+ * different GPUs (each holding part of every sequence's context) can be
+ * combined with pa_merge_partials after an all-gather.  (Split-KV across
+ * devices: the pages' engine shards attention by heads only; the key split
+ * and its log-sum-exp combination are the same as the in-GPU split of
+ * pa_decode, exact up to rounding.)
+ *
+ * Over the context_lens[b] keys that block_tables[b] names here:
+ *   o_part[b][h][:] = sum_j p_j V_j / sum_j p_j,   p_j = 2^(s_j - max s)
+ *   lse_part[b][h]  = log2 sum_j 2^(s_j),           s_j = scale*log2(e)*<q[b,h], K_j>
+ * A sequence with no keys here gets o_part = 0 and lse_part = -inf.
+ * o_part:   [num_seqs, num_heads, head_dim] fp32 (16-byte aligned).
+ * lse_part: [num_seqs, num_heads] fp32.
+ * Every other argument, the workspace rule and the errors are pa_decode's.
+ */
+PA_API pa_status pa_decode_partial(float* o_part, float* lse_part, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs, int32_t num_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                            float scale, int32_t kv_chunk_size, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
+ * pa_merge_partials -- combine num_partials partials of every row (one row
+ * per sequence and query head):
+ *   M = max_r lse_r,  out = sum_r 2^(lse_r - M) o_r / sum_r 2^(lse_r - M)
+ * rounded to bf16; a row whose partials all have lse = -inf is 0.
+ * o_parts:   [num_partials, num_rows, head_dim] fp32.
+ * lse_parts: [num_partials, num_rows] fp32.
+ * out:       [num_rows, head_dim] bf16.  head_dim 64 or 128.
+ */
+PA_API pa_status pa_merge_partials(void* out, const float* o_parts, const float* lse_parts, int32_t num_partials,
+                            int32_t num_rows, int32_t head_dim, void* stream);
 
 /*
  * pa_prefill_varlen -- varlen causal prefill against the paged cache.

@@ -31,6 +31,9 @@ _PROTOS = {
     "pa_prefill_varlen": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _i32, _i32, _i32, _i32,
                                          _i32, _i32, _i32, _f32, _i32, _vp]),
     "pa_device_error": (ctypes.c_int, [ctypes.POINTER(_i32), _vp]),
+    "pa_decode_partial": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32,
+                                         _i32, _i32, _f32, _i32, _vp, _sz, _vp]),
+    "pa_merge_partials": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, _vp]),
     "pa_rotary_cos_sin_cache": (ctypes.c_int, [_vp, _i32, _i32, ctypes.c_double, _vp]),
     "pa_rotary_store_kvcache": (ctypes.c_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _vp,
                                                _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
@@ -180,6 +183,58 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len, sca
                                block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
                                int(max_context_len), B, hq, hkv, d, bs, nb, float(scale), int(kv_chunk_size), ws_ptr,
                                ws_len, _stream(q, stream)), "pa_decode")
+    return out
+
+
+def decode_partial(q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, *, o_part=None,
+                   lse_part=None, workspace=None, kv_chunk_size=0, stream=None):
+    """pa_decode_partial: fp32 partial (o [B, Hq, D], lse [B, Hq] in log2 units) over the keys the tables name."""
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _cuda(t, n, torch.bfloat16)
+        _dense(t, n)
+    _cuda(block_tables, "block_tables", torch.int32)
+    _cuda(context_lens, "context_lens", torch.int32)
+    _dense(block_tables, "block_tables")
+    _dense(context_lens, "context_lens")
+    B, hq, d = q.shape
+    nb, bs, hkv, _ = k_cache.shape
+    if o_part is None:
+        o_part = torch.empty(B, hq, d, dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty(B, hq, dtype=torch.float32, device=q.device)
+    for n, t in (("o_part", o_part), ("lse_part", lse_part)):
+        _cuda(t, n, torch.float32)
+        _dense(t, n)
+    need = decode_workspace_size(B, hq, hkv, d, int(max_context_len), bs, kv_chunk_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(q.device):
+        _check(lib().pa_decode_partial(o_part.data_ptr(), lse_part.data_ptr(), q.data_ptr(), k_cache.data_ptr(),
+                                       v_cache.data_ptr(), block_tables.data_ptr(), block_tables.shape[1],
+                                       context_lens.data_ptr(), int(max_context_len), B, hq, hkv, d, bs, nb,
+                                       float(scale), kv_chunk_size, ws_ptr, ws_len, _stream(q, stream)),
+               "pa_decode_partial")
+    return o_part, lse_part
+
+
+def merge_partials(o_parts, lse_parts, *, out=None, stream=None):
+    """pa_merge_partials: o_parts [R, B, Hq, D] fp32 and lse_parts [R, B, Hq] fp32 -> out [B, Hq, D] bf16."""
+    _cuda(o_parts, "o_parts", torch.float32)
+    _cuda(lse_parts, "lse_parts", torch.float32)
+    _dense(o_parts, "o_parts")
+    _dense(lse_parts, "lse_parts")
+    R, B, hq, d = o_parts.shape
+    if tuple(lse_parts.shape) != (R, B, hq):
+        raise ValueError("lse_parts must be [R, B, Hq]")
+    if out is None:
+        out = torch.empty(B, hq, d, dtype=torch.bfloat16, device=o_parts.device)
+    _cuda(out, "out", torch.bfloat16)
+    _dense(out, "out")
+    with torch.cuda.device(o_parts.device):
+        _check(lib().pa_merge_partials(out.data_ptr(), o_parts.data_ptr(), lse_parts.data_ptr(), R, B * hq, d,
+                                       _stream(o_parts, stream)), "pa_merge_partials")
     return out
 
 

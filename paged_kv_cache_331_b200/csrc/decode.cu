@@ -47,6 +47,8 @@ struct DecodeParams {
   const int32_t* context_lens;
   float* ws_acc;
   float* ws_ml;
+  float* o_part;            // partial mode: normalised fp32 output [B, Hq, D] instead of out
+  float* lse_part;          //               log2-sum-exp of the scaled scores [B, Hq]
   int32_t max_blocks_per_seq;
   int32_t max_context_len;
   int32_t num_heads;
@@ -152,10 +154,15 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
   const int L = clamp_context(__ldg(p.context_lens + b), p);
   const int hq0 = g * G;
 
-  if (L == 0) {   // no keys: the output is defined as zero
-    if (chunk == 0)
-      for (int i = threadIdx.x; i < G * D; i += kThreads)
-        p.out[(static_cast<int64_t>(b) * p.num_heads + hq0) * D + i] = __float2bfloat16(0.f);
+  if (L == 0) {   // no keys: the output is defined as zero (a partial: 0 with lse = -inf)
+    if (chunk == 0) {
+      const int64_t base = (static_cast<int64_t>(b) * p.num_heads + hq0) * D;
+      for (int i = threadIdx.x; i < G * D; i += kThreads) {
+        if (p.o_part) p.o_part[base + i] = 0.f;
+        else p.out[base + i] = __float2bfloat16(0.f);
+      }
+      if (p.lse_part && threadIdx.x < G) p.lse_part[static_cast<int64_t>(b) * p.num_heads + hq0 + threadIdx.x] = -INFINITY;
+    }
     return;
   }
   const int start = chunk * p.chunk_tokens;
@@ -376,7 +383,12 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
     }
     const int64_t row = static_cast<int64_t>(b) * p.num_heads + hq0 + h;
     if (nchunks == 1) {
-      p.out[row * D + d] = __float2bfloat16(o / lsum);
+      if (p.o_part) {
+        p.o_part[row * D + d] = o / lsum;
+        if (d == 0) p.lse_part[row] = M + log2f(lsum);
+      } else {
+        p.out[row * D + d] = __float2bfloat16(o / lsum);
+      }
     } else {
       const int64_t idx = row * p.max_chunks + chunk;
       p.ws_acc[idx * D + d] = o;
@@ -421,10 +433,55 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p,
     }
   }
   const float inv = 1.f / lsum;
+  if (p.o_part) {   // partial mode: keep the normalised output in fp32, with its log2-sum-exp
+    float* op = p.o_part + static_cast<int64_t>(row) * D + lane * DPV;
+#pragma unroll
+    for (int c = 0; c < DPV; ++c) op[c] = o[c] * inv;
+    if (lane == 0) p.lse_part[row] = M + log2f(lsum);
+    return;
+  }
   __nv_bfloat16* out = p.out + static_cast<int64_t>(row) * D + lane * DPV;
 #pragma unroll
   for (int c = 0; c < DPV; c += 2)
     *reinterpret_cast<uint32_t*>(out + c) = pack_bf16x2(o[c] * inv, o[c + 1] * inv);
+}
+
+// Combination of R partials per (sequence, head) row (one warp per row):
+//   M = max_r lse_r,  out = sum_r 2^(lse_r - M) o_r / sum_r 2^(lse_r - M)
+// (a row whose partials all hold no keys, lse = -inf everywhere, is 0).
+template <int D>
+__global__ void __launch_bounds__(128) merge_lse_kernel(__nv_bfloat16* __restrict__ out,
+                                                        const float* __restrict__ o_parts,
+                                                        const float* __restrict__ lse_parts, int32_t num_parts,
+                                                        int32_t num_rows) {
+  constexpr int DPV = D / 32;
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= num_rows) return;
+  float M = -INFINITY;
+  for (int r = lane; r < num_parts; r += 32) M = fmaxf(M, __ldg(lse_parts + static_cast<int64_t>(r) * num_rows + row));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float o[DPV];
+#pragma unroll
+  for (int c = 0; c < DPV; ++c) o[c] = 0.f;
+  float wsum = 0.f;
+  if (M != -INFINITY) {
+    for (int r = 0; r < num_parts; ++r) {
+      const float l = __ldg(lse_parts + static_cast<int64_t>(r) * num_rows + row);
+      if (l == -INFINITY) continue;
+      const float w = fast_exp2(l - M);
+      wsum += w;
+      const float* src = o_parts + (static_cast<int64_t>(r) * num_rows + row) * D + lane * DPV;
+#pragma unroll
+      for (int c = 0; c < DPV; ++c) o[c] += w * __ldg(src + c);
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat16* dst = out + static_cast<int64_t>(row) * D + lane * DPV;
+#pragma unroll
+  for (int c = 0; c < DPV; c += 2)
+    *reinterpret_cast<uint32_t*>(dst + c) = pack_bf16x2(o[c] * inv, o[c + 1] * inv);
 }
 
 template <int D, int G>
@@ -505,6 +562,8 @@ pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.context_lens = a.context_lens;
   p.ws_acc = a.ws_acc;
   p.ws_ml = a.ws_ml;
+  p.o_part = a.o_part;
+  p.lse_part = a.lse_part;
   p.max_blocks_per_seq = a.max_blocks_per_seq;
   p.max_context_len = a.max_context_len;
   p.num_heads = a.num_heads;
@@ -531,6 +590,22 @@ pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     return PA_ERR_CUDA;
   }
   return PA_OK;
+}
+
+}  // namespace pa
+
+namespace pa {
+
+cudaError_t launch_merge_lse(void* out, const float* o_parts, const float* lse_parts, int32_t num_parts,
+                             int32_t num_rows, int32_t head_dim, cudaStream_t stream) {
+  const unsigned blocks = static_cast<unsigned>((num_rows + 3) / 4);
+  if (head_dim == 128)
+    merge_lse_kernel<128><<<blocks, 128, 0, stream>>>(static_cast<__nv_bfloat16*>(out), o_parts, lse_parts,
+                                                      num_parts, num_rows);
+  else
+    merge_lse_kernel<64><<<blocks, 128, 0, stream>>>(static_cast<__nv_bfloat16*>(out), o_parts, lse_parts,
+                                                     num_parts, num_rows);
+  return cudaGetLastError();
 }
 
 }  // namespace pa

@@ -275,12 +275,15 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num
   return workspace_bytes_for(num_seqs, num_heads, head_dim, chunks_for(max_context_len, chunk));
 }
 
-pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
-                    int32_t max_context_len, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
-                    int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t kv_chunk_size,
-                    void* workspace, size_t workspace_bytes, void* stream) {
+// pa_decode and pa_decode_partial: out (bf16) or the fp32 partials (o_part, lse_part).
+static pa_status decode_common(const char* who, void* out, float* o_part, float* lse_part, const void* q,
+                               const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                               int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t max_context_len,
+                               int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t block_size, int32_t num_blocks, float scale, int32_t kv_chunk_size,
+                               void* workspace, size_t workspace_bytes, void* stream) {
   t_last_error[0] = 0;
+  const bool partial = o_part != nullptr || lse_part != nullptr;
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "decode: num_seqs < 0");
   pa_status st = check_cache_shape("decode", num_heads, num_kv_heads, head_dim, block_size, num_blocks);
   if (st != PA_OK) return st;
@@ -290,10 +293,11 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     return fail(PA_ERR_INVALID_ARG, "decode: kv_chunk_size must be 0 or a positive multiple of %d", kDecodeTile);
   if (!(scale > 0.f) || !isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "decode: scale must be finite and > 0");
   if (num_seqs == 0) return PA_OK;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
-    return fail(PA_ERR_INVALID_ARG, "decode: null pointer");
-  if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache))
-    return fail(PA_ERR_INVALID_ARG, "decode: q, out, k_cache and v_cache must be 16-byte aligned");
+  if ((partial ? (!o_part || !lse_part) : !out) || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PA_ERR_INVALID_ARG, "%s: null pointer", who);
+  if (!aligned16(q) || !aligned16(partial ? static_cast<const void*>(o_part) : out) || !aligned16(k_cache) ||
+      !aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG, "%s: q, the output and the caches must be 16-byte aligned", who);
   if (static_cast<int64_t>(num_seqs) > 65535) return fail(PA_ERR_UNSUPPORTED, "decode: more than 65535 sequences");
   const int32_t chunk = resolve_chunk(num_seqs, num_kv_heads, max_context_len, kv_chunk_size);
   const int32_t nchunks = chunks_for(max_context_len, chunk);
@@ -303,6 +307,8 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                 workspace ? workspace_bytes : (size_t)0);
   DecodeArgs a;
   a.out = out;
+  a.o_part = o_part;
+  a.lse_part = lse_part;
   a.q = q;
   a.k_cache = k_cache;
   a.v_cache = v_cache;
@@ -325,6 +331,49 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   a.max_chunks = nchunks;
   a.scale = scale;
   return launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                    int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t kv_chunk_size,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_common("decode", out, nullptr, nullptr, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                       context_lens, max_context_len, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                       num_blocks, scale, kv_chunk_size, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_partial(float* o_part, float* lse_part, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs, int32_t num_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                            float scale, int32_t kv_chunk_size, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!o_part || !lse_part) {
+    t_last_error[0] = 0;
+    if (num_seqs == 0) return PA_OK;
+    return fail(PA_ERR_INVALID_ARG, "decode_partial: null o_part or lse_part");
+  }
+  return decode_common("decode_partial", nullptr, o_part, lse_part, q, k_cache, v_cache, block_tables,
+                       max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads, num_kv_heads,
+                       head_dim, block_size, num_blocks, scale, kv_chunk_size, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_merge_partials(void* out, const float* o_parts, const float* lse_parts, int32_t num_partials,
+                            int32_t num_rows, int32_t head_dim, void* stream) {
+  t_last_error[0] = 0;
+  if (num_partials <= 0 || num_rows < 0) return fail(PA_ERR_INVALID_ARG, "merge_partials: need num_partials > 0");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "merge_partials: head_dim %d not supported (64 or 128)", head_dim);
+  if (num_rows == 0) return PA_OK;
+  if (!out || !o_parts || !lse_parts) return fail(PA_ERR_INVALID_ARG, "merge_partials: null pointer");
+  if ((reinterpret_cast<uintptr_t>(out) & 3u) || (reinterpret_cast<uintptr_t>(o_parts) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse_parts) & 3u))
+    return fail(PA_ERR_INVALID_ARG, "merge_partials: pointers must be 4-byte aligned");
+  cudaError_t e = launch_merge_lse(out, o_parts, lse_parts, num_partials, num_rows, head_dim,
+                                   static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "merge_partials launch: %s", cudaGetErrorString(e));
+  return PA_OK;
 }
 
 pa_status pa_prefill_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,

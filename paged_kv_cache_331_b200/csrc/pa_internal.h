@@ -71,6 +71,8 @@ struct DecodeArgs {
   const int32_t* context_lens;
   float* ws_acc;            // [B, Hq, max_chunks, D] (unused when max_chunks == 1)
   float* ws_ml;             // [B, Hq, max_chunks, 2]
+  float* o_part;            // non-null: write fp32 partials (o, lse) instead of out
+  float* lse_part;
   int32_t max_blocks_per_seq;
   int32_t max_context_len;
   int32_t num_seqs;
@@ -88,6 +90,8 @@ constexpr int kDecodeTile = 64;   // tokens per decode pipeline stage
 
 int32_t decode_auto_chunk(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int sm_count);
 pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_merge_lse(void* out, const float* o_parts, const float* lse_parts, int32_t num_parts,
+                             int32_t num_rows, int32_t head_dim, cudaStream_t stream);
 
 // ---------------------------------------------------------------- prefill --
 struct PrefillArgs {
