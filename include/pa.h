@@ -234,6 +234,30 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache
                                    int32_t num_blocks, float scale, int32_t kv_chunk_size, void* stream);
 
 /*
+ * pa_store_decode -- pa_store_kvcache of one new token per sequence followed
+ * by pa_decode, in one launch.  ("Nano-vLLM 源碼學習" §二.2: in decode the
+ * attention layer stores the new token's k and v, then attends over the cache;
+ * "Architektur im Überblick", CUDA Graph Optimierung: fewer launches per
+ * decode step.)
+ *
+ * key, value: [num_seqs, num_kv_heads, head_dim] bf16 with row strides in
+ * elements, as for pa_store_kvcache; slot_mapping: [num_seqs] int32.  Token b
+ * is the newest token of sequence b: slot_mapping[b] must be -1 (nothing is
+ * stored) or the slot of position context_lens[b]-1 in block_tables[b].  The
+ * CTA that reads that position writes the row first, so the result equals
+ * the two separate calls.  Any other slot is not written and sets device
+ * error code 5.  key/value rows must be 16-byte aligned with strides that are
+ * multiples of 8 elements (PA_ERR_UNSUPPORTED otherwise).  Every other
+ * argument, the workspace rule and the errors are pa_decode's.
+ */
+PA_API pa_status pa_store_decode(void* out, const void* q, const void* key, const void* value, int64_t key_row_stride,
+                          int64_t value_row_stride, const int32_t* slot_mapping, void* k_cache, void* v_cache,
+                          const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                          int32_t max_context_len, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                          int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+                          int32_t kv_chunk_size, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * pa_decode_partial -- pa_decode over the keys this caller holds, returning
  * an fp32 partial instead of the bf16 output, so that partials computed on
  * different GPUs (each holding part of every sequence's context) can be
@@ -305,7 +329,8 @@ PA_API pa_status pa_prefill_varlen(void* out, const void* q, const void* k_cache
  * and pa_rotary_store_kvcache sets it for a position outside its table.
  * Codes: 0 none, 1 a pipeline wait timed out, 2 the wait for in-flight copies
  * at exit timed out, 3 dynamic shared memory misaligned, 4 rotary position
- * out of range.  Diagnostic only.
+ * out of range, 5 a pa_store_decode slot that is not the new token's.
+ * Diagnostic only.
  */
 PA_API pa_status pa_device_error(int32_t* code_out, void* stream);
 

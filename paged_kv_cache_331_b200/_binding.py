@@ -34,6 +34,8 @@ _PROTOS = {
     "pa_decode_partial": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32,
                                          _i32, _i32, _f32, _i32, _vp, _sz, _vp]),
     "pa_merge_partials": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, _vp]),
+    "pa_store_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32,
+                                       _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp]),
     "pa_rotary_cos_sin_cache": (ctypes.c_int, [_vp, _i32, _i32, ctypes.c_double, _vp]),
     "pa_rotary_store_kvcache": (ctypes.c_int, [_vp, _vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _vp, _vp, _vp,
                                                _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
@@ -183,6 +185,37 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len, sca
                                block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
                                int(max_context_len), B, hq, hkv, d, bs, nb, float(scale), int(kv_chunk_size), ws_ptr,
                                ws_len, _stream(q, stream)), "pa_decode")
+    return out
+
+
+def store_decode(q, key, value, slot_mapping, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, *,
+                 out=None, workspace=None, kv_chunk_size=0, stream=None):
+    """pa_store_decode: store each sequence's new K/V row (slot of position L-1, or -1) and decode, one launch."""
+    for n, t in (("q", q), ("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _cuda(t, n, torch.bfloat16)
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _dense(t, n)
+    for n, t in (("slot_mapping", slot_mapping), ("block_tables", block_tables), ("context_lens", context_lens)):
+        _cuda(t, n, torch.int32)
+        _dense(t, n)
+    B, hq, d = q.shape
+    nb, bs, hkv, _ = k_cache.shape
+    for name, t in (("key", key), ("value", value)):
+        if t.shape[0] != B or tuple(t.shape[1:]) != (hkv, d) or t.stride(-1) != 1 or t.stride(-2) != d:
+            raise ValueError(f"{name} must be [B, {hkv}, {d}] with dense rows")
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_size(B, hq, hkv, d, int(max_context_len), bs, kv_chunk_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(q.device):
+        _check(lib().pa_store_decode(out.data_ptr(), q.data_ptr(), key.data_ptr(), value.data_ptr(), key.stride(0),
+                                     value.stride(0), slot_mapping.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                     block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+                                     int(max_context_len), B, hq, hkv, d, bs, nb, float(scale), kv_chunk_size, ws_ptr,
+                                     ws_len, _stream(q, stream)), "pa_store_decode")
     return out
 
 

@@ -26,6 +26,8 @@
 //    (m, l, acc) at the end through shared memory.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include <math.h>
 
 #include "pa_device.cuh"
@@ -39,6 +41,16 @@ constexpr int kWarps = 4;                  // consumer warps
 constexpr int kTPW = kTile / kWarps;       // tokens per consumer warp per tile
 constexpr int kRounds = kTPW / 4;          // QK rounds (4 tokens per warp per round)
 constexpr int kThreads = (kWarps + 1) * 32;
+
+// Split-KV merge inside the split kernel: each launch uses one of
+// kMergeSlots arrays of per-(sequence, kv head) counters; the CTA whose
+// increment completes the count merges every chunk's partial and puts the
+// counter back to zero for the next launch that uses the slot.  The host
+// rotates slots between launches, so launches in flight at the same time on
+// different streams do not share one.
+constexpr int kMergeSlots = 16;
+constexpr int kMergeCounters = 16384;   // sequences x kv heads per launch; above it a merge kernel runs
+__device__ unsigned int g_decode_merge_cnt[kMergeSlots][kMergeCounters];
 
 struct DecodeParams {
   __nv_bfloat16* out;
@@ -58,6 +70,17 @@ struct DecodeParams {
   int32_t max_chunks;
   float scale_log2;
   unsigned int* err;
+  int32_t num_kv_heads;
+  int32_t merge_slot;       // >= 0: the last chunk CTA merges (counters of this slot); -1: merge kernel
+  int32_t o_stride;         // head_dim (row stride of out / o_part)
+  // fused store (slot_mapping != null): new K/V rows [num_seqs, Hkv, D] with row strides in elements
+  const __nv_bfloat16* new_k;
+  const __nv_bfloat16* new_v;
+  int64_t new_k_stride;
+  int64_t new_v_stride;
+  const int32_t* slot_mapping;
+  __nv_bfloat16* k_cache;
+  __nv_bfloat16* v_cache;
 };
 
 // Per-shape configuration.  Two CTAs share an SM whenever their shared memory
@@ -79,6 +102,17 @@ struct DecodeCfg {
   static_assert(merge_bytes <= kStages * kv_stage_elems * 2, "merge area must fit in the K stages");
   static_assert(bar_off % 8 == 0, "alignment");
 };
+
+// One output element of a finished row: bf16 out, or in partial mode the
+// normalised fp32 value (and, once per row, its log2-sum-exp).
+__device__ __forceinline__ void write_row(const DecodeParams& p, int64_t row, int d, float o, float M, float lsum) {
+  if (p.o_part) {
+    p.o_part[row * (p.o_stride) + d] = o / lsum;
+    if (d == 0) p.lse_part[row] = M + log2f(lsum);
+  } else {
+    p.out[row * p.o_stride + d] = __float2bfloat16(o / lsum);
+  }
+}
 
 __device__ __forceinline__ int clamp_context(int L, const DecodeParams& p) {
   L = min(L, p.max_context_len);
@@ -182,6 +216,32 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
 
   if (warp == kWarps) {
     // ------------------------------------------------------------ producer --
+    if (p.slot_mapping && chunk == nchunks - 1) {
+      // Fused store: this CTA is the only reader of position L-1 (its last
+      // tile), so it writes the new token's K/V row of kv head g into the
+      // cache before loading any tile.  The slot must be that position's;
+      // any other slot (but -1) is reported and not written.
+      const int32_t slot = __ldg(p.slot_mapping + b);
+      const int32_t* btb = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+      const int pos = L - 1;
+      const int64_t expect = static_cast<int64_t>(__ldg(btb + pos / p.block_size)) * p.block_size + pos % p.block_size;
+      if (slot >= 0 && slot == expect) {
+        constexpr int kLanesPerRow = D / 8;   // 16-byte pieces of one head row
+        if (lane < 2 * kLanesPerRow) {
+          const bool is_v = lane >= kLanesPerRow;
+          const int piece = is_v ? lane - kLanesPerRow : lane;
+          const __nv_bfloat16* src = (is_v ? p.new_v + b * p.new_v_stride : p.new_k + b * p.new_k_stride) +
+                                     static_cast<int64_t>(g) * D + piece * 8;
+          __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) +
+                               (static_cast<int64_t>(slot) * p.num_kv_heads + g) * D + piece * 8;
+          *reinterpret_cast<uint4*>(dst) = ld_nc_v4(src);
+          fence_proxy_async_global();
+        }
+      } else if (slot != -1 && lane == 0) {
+        record_error(p.err, kErrBadSlot);
+      }
+      __syncwarp();
+    }
     if (lane == 0) {
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
@@ -383,12 +443,7 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
     }
     const int64_t row = static_cast<int64_t>(b) * p.num_heads + hq0 + h;
     if (nchunks == 1) {
-      if (p.o_part) {
-        p.o_part[row * D + d] = o / lsum;
-        if (d == 0) p.lse_part[row] = M + log2f(lsum);
-      } else {
-        p.out[row * D + d] = __float2bfloat16(o / lsum);
-      }
+      write_row(p, row, d, o, M, lsum);
     } else {
       const int64_t idx = row * p.max_chunks + chunk;
       p.ws_acc[idx * D + d] = o;
@@ -397,6 +452,36 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
         p.ws_ml[2 * idx + 1] = lsum;
       }
     }
+  }
+  if (nchunks == 1 || p.merge_slot < 0) return;
+
+  // ------------------------------------- the last chunk of (b, g) merges all --
+  __shared__ int s_last;
+  __threadfence();                       // this CTA's partials are visible device-wide
+  named_barrier_sync(1, kWarps * 32);
+  if (threadIdx.x == 0) {
+    unsigned int* cnt = &g_decode_merge_cnt[p.merge_slot][b * p.num_kv_heads + g];
+    const unsigned int prev = atomicAdd(cnt, 1u);
+    s_last = prev == static_cast<unsigned int>(nchunks - 1);
+    if (s_last) *cnt = 0u;               // every chunk has counted: ready for the next launch
+  }
+  named_barrier_sync(1, kWarps * 32);
+  if (!s_last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < G * D; i += kWarps * 32) {
+    const int h = i / D, d = i % D;
+    const int64_t row = static_cast<int64_t>(b) * p.num_heads + hq0 + h;
+    const float* ml = p.ws_ml + row * p.max_chunks * 2;
+    const float* ac = p.ws_acc + row * p.max_chunks * D + d;
+    float M = -INFINITY;
+    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, __ldcg(ml + 2 * c));
+    float lsum = 0.f, o = 0.f;
+    for (int c = 0; c < nchunks; ++c) {
+      const float f = fast_exp2(__ldcg(ml + 2 * c) - M);
+      lsum += __ldcg(ml + 2 * c + 1) * f;
+      o += __ldcg(ac + static_cast<int64_t>(c) * D) * f;
+    }
+    write_row(p, row, d, o, M, lsum);
   }
 }
 
@@ -573,11 +658,23 @@ pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.max_chunks = a.max_chunks;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.err = current_device_info()->error_word;
+  p.num_kv_heads = a.num_kv_heads;
+  p.o_stride = a.head_dim;
+  p.new_k = static_cast<const __nv_bfloat16*>(a.new_k);
+  p.new_v = static_cast<const __nv_bfloat16*>(a.new_v);
+  p.new_k_stride = a.new_k_stride;
+  p.new_v_stride = a.new_v_stride;
+  p.slot_mapping = a.slot_mapping;
+  p.k_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(a.k_cache));
+  p.v_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(a.v_cache));
+  static std::atomic<uint32_t> launches{0};
+  const bool fused_merge = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads <= kMergeCounters;
+  p.merge_slot = (a.max_chunks > 1 && fused_merge) ? static_cast<int32_t>(launches.fetch_add(1) % kMergeSlots) : -1;
   const dim3 grid(static_cast<unsigned>(a.max_chunks), static_cast<unsigned>(a.num_kv_heads),
                   static_cast<unsigned>(a.num_seqs));
   pa_status st = a.head_dim == 128 ? dispatch_group<128>(G, tmK, tmV, p, grid, stream)
                                    : dispatch_group<64>(G, tmK, tmV, p, grid, stream);
-  if (st != PA_OK || a.max_chunks <= 1) return st;
+  if (st != PA_OK || a.max_chunks <= 1 || p.merge_slot >= 0) return st;
   const int32_t rows_out = a.num_seqs * a.num_heads;
   const unsigned mblocks = static_cast<unsigned>((rows_out + 3) / 4);
   if (a.head_dim == 128)

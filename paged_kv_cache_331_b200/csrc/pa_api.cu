@@ -275,13 +275,24 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num
   return workspace_bytes_for(num_seqs, num_heads, head_dim, chunks_for(max_context_len, chunk));
 }
 
-// pa_decode and pa_decode_partial: out (bf16) or the fp32 partials (o_part, lse_part).
+// The store a fused call makes before decoding (none when slot_mapping is null).
+struct FusedStore {
+  const void* key = nullptr;
+  const void* value = nullptr;
+  int64_t key_row_stride = 0;
+  int64_t value_row_stride = 0;
+  const int32_t* slot_mapping = nullptr;
+};
+
+// pa_decode, pa_decode_partial and pa_store_decode: out (bf16) or the fp32
+// partials (o_part, lse_part), with an optional fused store.
 static pa_status decode_common(const char* who, void* out, float* o_part, float* lse_part, const void* q,
                                const void* k_cache, const void* v_cache, const int32_t* block_tables,
                                int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t max_context_len,
                                int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
                                int32_t block_size, int32_t num_blocks, float scale, int32_t kv_chunk_size,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+                               void* workspace, size_t workspace_bytes, void* stream,
+                               const FusedStore& fs = FusedStore()) {
   t_last_error[0] = 0;
   const bool partial = o_part != nullptr || lse_part != nullptr;
   if (num_seqs < 0) return fail(PA_ERR_INVALID_ARG, "decode: num_seqs < 0");
@@ -305,7 +316,21 @@ static pa_status decode_common(const char* who, void* out, float* o_part, float*
   if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
     return fail(PA_ERR_WORKSPACE, "decode: workspace of %zu bytes (16-byte aligned) required, got %zu", need,
                 workspace ? workspace_bytes : (size_t)0);
-  DecodeArgs a;
+  if (fs.slot_mapping) {
+    const int64_t row = static_cast<int64_t>(num_kv_heads) * head_dim;
+    if (!fs.key || !fs.value) return fail(PA_ERR_INVALID_ARG, "%s: null key or value", who);
+    if (fs.key_row_stride < row || fs.value_row_stride < row)
+      return fail(PA_ERR_INVALID_ARG, "%s: row strides must be >= num_kv_heads*head_dim", who);
+    if (!aligned16(fs.key) || !aligned16(fs.value) || fs.key_row_stride % 8 || fs.value_row_stride % 8)
+      return fail(PA_ERR_UNSUPPORTED, "%s: key/value rows must be 16-byte aligned (use pa_store_kvcache + pa_decode)",
+                  who);
+  }
+  DecodeArgs a{};
+  a.new_k = fs.key;
+  a.new_v = fs.value;
+  a.new_k_stride = fs.key_row_stride;
+  a.new_v_stride = fs.value_row_stride;
+  a.slot_mapping = fs.slot_mapping;
   a.out = out;
   a.o_part = o_part;
   a.lse_part = lse_part;
@@ -357,6 +382,28 @@ pa_status pa_decode_partial(float* o_part, float* lse_part, const void* q, const
   return decode_common("decode_partial", nullptr, o_part, lse_part, q, k_cache, v_cache, block_tables,
                        max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads, num_kv_heads,
                        head_dim, block_size, num_blocks, scale, kv_chunk_size, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_store_decode(void* out, const void* q, const void* key, const void* value, int64_t key_row_stride,
+                          int64_t value_row_stride, const int32_t* slot_mapping, void* k_cache, void* v_cache,
+                          const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                          int32_t max_context_len, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                          int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+                          int32_t kv_chunk_size, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!slot_mapping) {
+    t_last_error[0] = 0;
+    if (num_seqs == 0) return PA_OK;
+    return fail(PA_ERR_INVALID_ARG, "store_decode: null slot_mapping");
+  }
+  FusedStore fs;
+  fs.key = key;
+  fs.value = value;
+  fs.key_row_stride = key_row_stride;
+  fs.value_row_stride = value_row_stride;
+  fs.slot_mapping = slot_mapping;
+  return decode_common("store_decode", out, nullptr, nullptr, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                       context_lens, max_context_len, num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                       num_blocks, scale, kv_chunk_size, workspace, workspace_bytes, stream, fs);
 }
 
 pa_status pa_merge_partials(void* out, const float* o_parts, const float* lse_parts, int32_t num_partials,

@@ -17,6 +17,7 @@ enum DeviceErrorCode : unsigned int {
   kErrDrainTimeout = 2,    // waiting for in-flight copies at exit ran out of time
   kErrSmemAlign = 3,       // dynamic shared memory not 1024-byte aligned
   kErrBadPosition = 4,     // a rotary position outside [0, max_position)
+  kErrBadSlot = 5,         // fused store + decode: a slot that is not the new token's position
 };
 
 #ifndef PA_WAIT_LIMIT_NS
@@ -170,6 +171,12 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 // async-proxy (TMA / tcgen05) reads of the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order this thread's generic-proxy global-memory writes before later
+// async-proxy (TMA) reads of the same memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ------------------------------------------------------------------- tcgen05 --

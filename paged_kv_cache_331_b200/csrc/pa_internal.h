@@ -73,6 +73,11 @@ struct DecodeArgs {
   float* ws_ml;             // [B, Hq, max_chunks, 2]
   float* o_part;            // non-null: write fp32 partials (o, lse) instead of out
   float* lse_part;
+  const void* new_k;        // fused store (slot_mapping non-null): new rows written before decoding
+  const void* new_v;
+  int64_t new_k_stride;
+  int64_t new_v_stride;
+  const int32_t* slot_mapping;
   int32_t max_blocks_per_seq;
   int32_t max_context_len;
   int32_t num_seqs;

@@ -1,11 +1,12 @@
-"""CUDA-graph capture of the decode step ([rotary +] store_kvcache + decode).
+"""CUDA-graph capture of the decode step (store + decode, or rotary store + decode).
 
 "Architektur im Überblick", section "CUDA Graph Optimierung": the engine
 captures its decode step once per batch size in [1, 2, 4, 8] + [16, 32, ...,
 max_bs], in descending order and into one shared memory pool, and replays
 the smallest captured graph that holds the current batch.  This runner does
 the same for the attention step of one layer: the new tokens' K/V rows are
-scattered into the cache and every sequence attends over its blocks.  Given
+scattered into the cache and every sequence attends over its blocks (one
+launch, pa_store_decode).  Given
 a rotary cos/sin cache, the step first rotates q and the new keys to their
 positions ("Nano-vLLM 源碼學習", layers, 7 rotary_embedding.py), fused with the
 store, and decode reads the rotated q.
@@ -64,9 +65,11 @@ class DecodeGraphRunner:
         self._capture()
 
     def _step(self, bs):
-        if self.cos_sin_cache is None:
-            pa.store_kvcache(self.new_k[:bs], self.new_v[:bs], self.k_cache, self.v_cache, self.slot_mapping[:bs])
-            q = self.q[:bs]
+        if self.cos_sin_cache is None:     # one launch: the new rows are stored by the decode kernel itself
+            pa.store_decode(self.q[:bs], self.new_k[:bs], self.new_v[:bs], self.slot_mapping[:bs], self.k_cache,
+                            self.v_cache, self.block_tables[:bs], self.context_lens[:bs], self.max_context_len,
+                            self.scale, out=self.out[:bs], workspace=self.workspace, kv_chunk_size=self.kv_chunk_size)
+            return
         else:
             q = pa.rotary_store_kvcache(self.q[:bs], self.new_k[:bs], self.new_v[:bs], self.positions[:bs],
                                         self.cos_sin_cache, self.k_cache, self.v_cache, self.slot_mapping[:bs],
