@@ -621,11 +621,25 @@ int32_t decode_auto_chunk(int32_t num_seqs, int32_t num_kv_heads, int32_t max_co
   const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
   if (max_context_len <= kMinChunk || units <= 0) return ((max(max_context_len, 1) + kTile - 1) / kTile) * kTile;
   const int64_t want = static_cast<int64_t>(kWavesTarget) * 2 * sm_count;
+  if (units >= want) return ((max_context_len + kTile - 1) / kTile) * kTile;   // enough CTAs unsplit
   int64_t splits = (want + units - 1) / units;
   const int64_t max_splits = (max_context_len + kMinChunk - 1) / kMinChunk;
   splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);
-  const int64_t per = (max_context_len + splits - 1) / splits;
-  return static_cast<int32_t>(((per + kTile - 1) / kTile) * kTile);
+  // Among one split fewer or more, prefer the count whose chunks (whole
+  // tiles) cover the longest context with the least overhang: a short last
+  // chunk leaves its CTA idle for most of a wave (ties: more CTAs).
+  int64_t best_chunk = 0, best_waste = INT64_MAX;
+  for (int64_t s2 = splits + 1; s2 >= splits - 1; --s2) {
+    if (s2 < 1 || s2 > max_splits) continue;
+    const int64_t per = (max_context_len + s2 - 1) / s2;
+    const int64_t chunk = ((per + kTile - 1) / kTile) * kTile;
+    const int64_t waste = ((max_context_len + chunk - 1) / chunk) * chunk - max_context_len;
+    if (waste < best_waste) {
+      best_waste = waste;
+      best_chunk = chunk;
+    }
+  }
+  return static_cast<int32_t>(best_chunk);
 }
 
 pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
