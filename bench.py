@@ -299,19 +299,20 @@ def bench_decode(args, world, rank, dev, peaks):
     achieved = alg_bytes / (decode_ms / 1e3) / 1e9
     traffic = profiled_traffic("decode")
 
-    # end to end through host buffers: per step H2D of q, new K/V rows and the metadata, D2H of out
-    hq_, hnk, hnv = pinned(w.q, "bf16"), pinned(w.new_k, "bf16"), pinned(w.new_v, "bf16")
-    hs, hbt, hcl = pinned(w.slot_mapping, "i32"), pinned(w.block_tables, "i32"), pinned(w.context_lens, "i32")
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq_, hnk, hnv, hs, hbt, hcl))
-    d2h = hout.numel() * hout.element_size()
+    # end to end through host buffers: every step copies q, the new K/V rows and the metadata (one packed pinned
+    # buffer) to the device, runs the fused store + decode, and copies out back -- one CUDA graph
+    from paged_kv_cache_331_b200.graphs import HostDecodeStep
+    hstep = HostDecodeStep(kc, vc, w.num_seqs, w.num_heads, w.block_tables.shape[1], maxL, w.scale)
+    hin = hstep.inputs()
+    for name, arr in (("q", w.q), ("new_k", w.new_k), ("new_v", w.new_v)):
+        hin[name].view(torch.int16).copy_(torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)))
+    hin["slot_mapping"].copy_(torch.from_numpy(w.slot_mapping))
+    hin["block_tables"].copy_(torch.from_numpy(w.block_tables))
+    hin["context_lens"].copy_(torch.from_numpy(w.context_lens))
+    h2d, d2h = hstep.h2d_bytes, hstep.d2h_bytes
 
     def e2e_step():
-        q.copy_(hq_, non_blocking=True); nk.copy_(hnk, non_blocking=True); nv.copy_(hnv, non_blocking=True)
-        slots.copy_(hs, non_blocking=True); bt.copy_(hbt, non_blocking=True); cl.copy_(hcl, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
-        torch.cuda.current_stream(dev).synchronize()
+        hstep.run()
 
     for _ in range(min(args.warmup, 10)):
         e2e_step()

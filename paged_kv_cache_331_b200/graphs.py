@@ -131,3 +131,71 @@ class DecodeGraphRunner:
         bs = self.load(q, new_k, new_v, slot_mapping, block_tables, context_lens, positions)
         self.replay(bs)
         return self.out[:q.shape[0]]
+
+
+class HostDecodeStep:
+    """A decode step fed from and returned to host memory, as one CUDA graph.
+
+    The step's inputs (q, the new K/V rows, their slots, the block tables and
+    the context lengths) live in one pinned host buffer, so the graph is a single
+    host-to-device copy, the fused store + decode (pa_store_decode), and a single
+    device-to-host copy of the output.  The caller fills the host views returned
+    by ``inputs()`` and calls ``run()``.  The KV cache stays on the device; its
+    address is baked into the graph.
+    """
+
+    _ALIGN = 256
+
+    def __init__(self, k_cache, v_cache, num_seqs, num_heads, max_blocks_per_seq, max_context_len, scale,
+                 kv_chunk_size=0):
+        nb, bs, hkv, d = k_cache.shape
+        dev = k_cache.device
+        B, hq = num_seqs, num_heads
+        spec = [("q", (B, hq, d), torch.bfloat16), ("new_k", (B, hkv, d), torch.bfloat16),
+                ("new_v", (B, hkv, d), torch.bfloat16), ("slot_mapping", (B,), torch.int32),
+                ("block_tables", (B, max_blocks_per_seq), torch.int32), ("context_lens", (B,), torch.int32)]
+        offs, o = [], 0
+        for _, shape, dt in spec:
+            n = int(torch.tensor(shape).prod().item()) * torch.empty((), dtype=dt).element_size()
+            offs.append((o, n))
+            o = (o + n + self._ALIGN - 1) // self._ALIGN * self._ALIGN
+        self.h2d_bytes = o
+        self.host = torch.zeros(o, dtype=torch.uint8).pin_memory()
+        self.dev = torch.zeros(o, dtype=torch.uint8, device=dev)
+
+        def views(buf):
+            return {name: buf[a:a + n].view(dt).view(shape) for (name, shape, dt), (a, n) in zip(spec, offs)}
+
+        self._h, self._d = views(self.host), views(self.dev)
+        self.out = torch.empty(B, hq, d, dtype=torch.bfloat16, device=dev)
+        self.host_out = torch.empty(B, hq, d, dtype=torch.bfloat16).pin_memory()
+        self.d2h_bytes = self.host_out.numel() * self.host_out.element_size()
+        ws = pa.decode_workspace_size(B, hq, hkv, d, max_context_len, bs, kv_chunk_size)
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.max_context_len, self.scale, self.kv_chunk_size = max_context_len, scale, kv_chunk_size
+        self._h["slot_mapping"].fill_(-1)            # an unfilled step stores nothing and reads nothing
+        self._h["block_tables"].fill_(-1)
+        self._step()                                   # eager once: kernel set-up happens outside the capture
+        torch.cuda.synchronize(dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self._step()
+
+    def _step(self):
+        d = self._d
+        self.dev.copy_(self.host, non_blocking=True)
+        pa.store_decode(d["q"], d["new_k"], d["new_v"], d["slot_mapping"], self.k_cache, self.v_cache,
+                        d["block_tables"], d["context_lens"], self.max_context_len, self.scale, out=self.out,
+                        workspace=self.workspace, kv_chunk_size=self.kv_chunk_size)
+        self.host_out.copy_(self.out, non_blocking=True)
+
+    def inputs(self):
+        """Host views to fill before run(): q, new_k, new_v, slot_mapping, block_tables, context_lens."""
+        return self._h
+
+    def run(self):
+        """Replay the step and wait for it; returns the host output [B, Hq, D] (bf16, pinned)."""
+        self.graph.replay()
+        torch.cuda.current_stream(self.out.device).synchronize()
+        return self.host_out

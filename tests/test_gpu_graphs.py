@@ -67,3 +67,29 @@ def test_rotary_graph_replay_matches_eager_and_oracle(oracle, n):
     _, ref = oracle.decode(q_rot, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
     assert_attention_close(out_g, ref, what=f"rotary graph replay n={n}")
     assert pa.device_error() == 0
+
+
+def test_host_decode_step_matches_the_device_calls(oracle):
+    from paged_kv_cache_331_b200.graphs import HostDecodeStep
+    rng = np.random.default_rng(77)
+    lens = rng.integers(1, 3000, 12).astype(np.int32)
+    w = W.decode_workload(lens, 16, 8, 128, 256, rng=rng)
+    a, b = DeviceDecode(w), DeviceDecode(w)
+    step = HostDecodeStep(a.k_cache, a.v_cache, 12, 16, w.block_tables.shape[1], 3072, w.scale)
+    h = step.inputs()
+    for name, arr in (("q", w.q), ("new_k", w.new_k), ("new_v", w.new_v)):
+        h[name].view(torch.int16).copy_(torch.from_numpy(arr.view(np.int16)))
+    h["slot_mapping"].copy_(torch.from_numpy(w.slot_mapping))
+    h["block_tables"].copy_(torch.from_numpy(w.block_tables))
+    h["context_lens"].copy_(torch.from_numpy(w.context_lens))
+    out_h = step.run().clone()
+    ref = pa.store_decode(b.q, b.new_k, b.new_v, b.slot_mapping, b.k_cache, b.v_cache, b.block_tables,
+                          b.context_lens, 3072, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h.view(torch.int16), ref.cpu().view(torch.int16))
+    assert torch.equal(a.k_cache.view(torch.int16), b.k_cache.view(torch.int16))
+    assert torch.equal(step.run().view(torch.int16), out_h.view(torch.int16))   # a second replay
+    oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
+    _, f64 = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
+    assert_attention_close(out_h, f64, what="host decode step")
+    assert pa.device_error() == 0
