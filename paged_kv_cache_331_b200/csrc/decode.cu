@@ -456,18 +456,24 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
   if (nchunks == 1 || p.merge_slot < 0) return;
 
   // ------------------------------------- the last chunk of (b, g) merges all --
+  // The barrier orders every consumer's partial writes before thread 0's
+  // device-scope fence (fences are cumulative), which publishes them before
+  // its increment; the last CTA's fence after its increment orders the
+  // partials of the other chunks before the reads that follow the barrier.
   __shared__ int s_last;
-  __threadfence();                       // this CTA's partials are visible device-wide
   named_barrier_sync(1, kWarps * 32);
   if (threadIdx.x == 0) {
+    __threadfence();
     unsigned int* cnt = &g_decode_merge_cnt[p.merge_slot][b * p.num_kv_heads + g];
     const unsigned int prev = atomicAdd(cnt, 1u);
     s_last = prev == static_cast<unsigned int>(nchunks - 1);
-    if (s_last) *cnt = 0u;               // every chunk has counted: ready for the next launch
+    if (s_last) {
+      *cnt = 0u;                         // every chunk has counted: ready for the next launch
+      __threadfence();
+    }
   }
   named_barrier_sync(1, kWarps * 32);
   if (!s_last) return;
-  __threadfence();
   for (int i = threadIdx.x; i < G * D; i += kWarps * 32) {
     const int h = i / D, d = i % D;
     const int64_t row = static_cast<int64_t>(b) * p.num_heads + hq0 + h;
