@@ -337,6 +337,20 @@ def bench_decode(args, world, rank, dev, peaks):
     }
 
 
+class L2Flush:
+    """Flush between timed reps: write a buffer larger than L2 (126 MB), then read another one, so that the
+    write-back of the flush's dirty lines happens before the timed region rather than inside it."""
+
+    def __init__(self, dev, nbytes=256 << 20):
+        import torch
+        self.w = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(nbytes // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        return self.r.sum()
+
+
 def bench_prefill(args, dev, peaks):
     import torch
     import paged_kv_cache_331_b200 as pa
@@ -348,7 +362,7 @@ def bench_prefill(args, dev, peaks):
     slots, bt = to_dev(w.slot_mapping, "i32", dev), to_dev(w.block_tables, "i32", dev)
     cq, ck = to_dev(w.cu_seqlens_q, "i32", dev), to_dev(w.cu_seqlens_k, "i32", dev)
     out = torch.empty_like(q)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2, written between reps
+    flush = L2Flush(dev)
 
     def store():
         pa.store_kvcache(nk, nv, kc, vc, slots)
@@ -362,7 +376,7 @@ def bench_prefill(args, dev, peaks):
     reps = max(3, min(args.steps, 100))
     st, pf = [], []
     for _ in range(reps):
-        flush.zero_()
+        flush()
         a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         a.record(); store(); b.record(); prefill(); c.record()
         st.append((a, b)); pf.append((b, c))
@@ -375,9 +389,11 @@ def bench_prefill(args, dev, peaks):
     store_bytes = 2 * 2 * int(w.cu_seqlens_q[-1]) * w.num_kv_heads * w.head_dim * 2 + 4 * int(w.cu_seqlens_q[-1])
     store_gbs = store_bytes / (store_ms / 1e3) / 1e9
     rot = bench_rotary_store(w, dev, q, nk, nv, kc, vc, slots, flush, reps)
+    big = bench_store_large(dev, reps)
     peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     return {
         "workload": w.name, "num_seqs": w.num_seqs, "prefix_len": 1024, "suffix": "U[64,512]",
+        "l2": "flushed before every rep: a 256 MB buffer written, then another 256 MB read",
         "total_q": int(w.cu_seqlens_q[-1]), "ms": prefill_ms, "flops": flops, "tflops": tflops,
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": tflops / peak_tf, "traffic": profiled_traffic("prefill"),
@@ -385,13 +401,45 @@ def bench_prefill(args, dev, peaks):
         "store": {"rows": int(w.cu_seqlens_q[-1]), "ms": store_ms, "gbs": store_gbs,
                   "frac": store_gbs / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "bytes": store_bytes},
         "rotary_store": rot,
+        "store_large": big,
         "gpu_launches_per_rep": 2,
     }
 
 
+def bench_store_large(dev, reps):
+    """store_kvcache of 65 536 new rows of the large-batch layer shape (8 kv heads, head_dim 128): 256 MB read and
+    256 MB written, more than L2 holds, so consecutive reps stream from HBM."""
+    import torch
+    import paged_kv_cache_331_b200 as pa
+    n, hkv, d, bs = 65536, 8, 128, 256
+    rng = np.random.default_rng(9)
+    key = torch.randn(n, hkv, d, dtype=torch.bfloat16, device=dev)
+    value = torch.randn(n, hkv, d, dtype=torch.bfloat16, device=dev)
+    nb = n // bs + 16
+    kc = torch.empty(nb, bs, hkv, d, dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    slots = torch.from_numpy(rng.permutation(nb * bs)[:n].astype(np.int32)).to(dev)
+    for _ in range(3):
+        pa.store_kvcache(key, value, kc, vc, slots)
+    torch.cuda.synchronize(dev)
+    ev = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(); pa.store_kvcache(key, value, kc, vc, slots); b.record()
+        ev.append((a, b))
+    torch.cuda.synchronize(dev)
+    assert pa.device_error() == 0
+    ms = float(np.median([x.elapsed_time(y) for x, y in ev]))
+    nbytes = 2 * 2 * n * hkv * d * 2 + 4 * n
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"rows": n, "ms": ms, "bytes": nbytes, "gbs": gbs,
+            "frac": gbs / load_peaks().get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+            "note": "inputs larger than L2; random unique slots"}
+
+
 def bench_rotary_store(w, dev, q, nk, nv, kc, vc, slots, flush, reps):
     """The prefill's new tokens through the fused rotary + store kernel (q rotated into a new buffer, rotated keys
-    and values into the cache), L2 flushed between reps."""
+    and values into the cache), L2 flushed (written, then evicted by a read) between reps."""
     import torch
     import paged_kv_cache_331_b200 as pa
     n = int(w.cu_seqlens_q[-1])
@@ -407,7 +455,7 @@ def bench_rotary_store(w, dev, q, nk, nv, kc, vc, slots, flush, reps):
     torch.cuda.synchronize(dev)
     ev = []
     for _ in range(reps):
-        flush.zero_()
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(); pa.rotary_store_kvcache(q, nk, nv, pos, table, kc, vc, slots, out=q_rot); b.record()
         ev.append((a, b))
