@@ -106,3 +106,15 @@ def test_decode_workspace_too_small_is_rejected():
 
 def test_decode_no_device_error():
     assert pa.device_error() == 0
+
+
+def test_decode_empty_batch():
+    q = torch.empty(0, 4, 64, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(2, 16, 2, 64, dtype=torch.bfloat16, device="cuda")
+    bt = torch.empty(0, 1, dtype=torch.int32, device="cuda")
+    cl = torch.empty(0, dtype=torch.int32, device="cuda")
+    out = pa.decode(q, kc, kc, bt, cl, 0, 0.125)
+    o, lse = pa.decode_partial(q, kc, kc, bt, cl, 0, 0.125)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 4, 64) and o.shape == (0, 4, 64) and lse.shape == (0, 4)
+    assert pa.device_error() == 0

@@ -92,3 +92,26 @@ def test_prefill_poisoned_cache(oracle):
 
 def test_prefill_no_device_error():
     assert pa.device_error() == 0
+
+
+def test_prefill_fully_cached_sequences_and_empty_batch(oracle):
+    """A sequence whose prompt is entirely cached has no query rows (Lq = 0); the others are unaffected, and a
+    batch with no query rows at all launches nothing."""
+    rng = np.random.default_rng(31)
+    w = W.prefill_workload(32, [0, 5, 0, 70], 8, 2, 128, 16, rng=rng)
+    dw = DevicePrefill(w)
+    pa.store_kvcache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping)
+    out = pa.prefill_varlen(dw.q, dw.k_cache, dw.v_cache, dw.cu_seqlens_q, dw.cu_seqlens_k, w.max_seqlen_q,
+                            w.max_seqlen_k, dw.block_tables, w.scale, True)
+    torch.cuda.synchronize()
+    oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
+    _, ref = oracle.prefill_varlen(w.q, w.k_cache, w.v_cache, w.cu_seqlens_q, w.cu_seqlens_k, w.block_tables,
+                                   w.scale, True, want_f64=True)
+    assert_attention_close(out, ref, what="prefill with fully cached sequences")
+    w0 = W.prefill_workload(32, [0, 0], 8, 2, 128, 16, rng=rng)
+    d0 = DevicePrefill(w0)
+    out0 = pa.prefill_varlen(d0.q, d0.k_cache, d0.v_cache, d0.cu_seqlens_q, d0.cu_seqlens_k, w0.max_seqlen_q,
+                             w0.max_seqlen_k, d0.block_tables, w0.scale, True)
+    torch.cuda.synchronize()
+    assert out0.shape[0] == 0
+    assert pa.device_error() == 0
