@@ -77,8 +77,11 @@ class BlockManager:
     def __del__(self):
         h = getattr(self, "_h", None)
         if h:
-            _lib().pa_bm_destroy(h)
             self._h = None
+            try:
+                _lib().pa_bm_destroy(h)
+            except Exception:     # interpreter shutdown: the library may already be gone
+                pass
 
     def _ok(self, status, what):
         _binding._check(status, what)

@@ -22,6 +22,7 @@ supplies the graph objects, buffers and streams.
 from __future__ import annotations
 
 import bisect
+import math
 
 import torch
 
@@ -156,7 +157,7 @@ class HostDecodeStep:
                 ("block_tables", (B, max_blocks_per_seq), torch.int32), ("context_lens", (B,), torch.int32)]
         offs, o = [], 0
         for _, shape, dt in spec:
-            n = int(torch.tensor(shape).prod().item()) * torch.empty((), dtype=dt).element_size()
+            n = math.prod(shape) * torch.empty((), dtype=dt).element_size()
             offs.append((o, n))
             o = (o + n + self._ALIGN - 1) // self._ALIGN * self._ALIGN
         self.h2d_bytes = o
