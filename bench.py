@@ -26,6 +26,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import platform
 import math
 import os
 import re
@@ -539,9 +540,25 @@ def cpu_baseline(w, budget_s=12.0):
         orc.decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale)
         t_total += time.perf_counter() - t
         reps += 1
+    # the same oracle on one thread, one rep of the decode (about a second)
+    t = time.perf_counter()
+    orc.decode(w.q, kc, vc, w.block_tables, w.context_lens, w.scale, nthreads=1)
+    t1 = time.perf_counter() - t
     return {"value": kv_bytes * reps / t_total / 1e9, "unit": "GB/s", "cores": orc.max_threads(), "kind": "oracle",
             "sample": f"full workload (store + decode of all {w.num_seqs} sequences), {reps} rep(s), "
-                      f"{t_total:.1f} s", "seconds": t_total}
+                      f"{t_total:.1f} s", "seconds": t_total, "cpu_model": cpu_model(),
+            "one_thread": {"value": kv_bytes / t1 / 1e9, "unit": "GB/s", "sample": "one decode of the full workload",
+                           "seconds": t1}}
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
 
 
 def run_ours(args, world, rank, local):
@@ -585,6 +602,7 @@ def run_ours(args, world, rank, local):
         line["graph"] = gr
     if cpu is not None:
         line["cpu_baseline"] = cpu
+        line["speedup_vs_cpu_baseline"] = round(d["value"] / cpu["value"], 1)
     print(json.dumps(line), flush=True)
 
 
