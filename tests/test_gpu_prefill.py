@@ -115,3 +115,27 @@ def test_prefill_fully_cached_sequences_and_empty_batch(oracle):
     torch.cuda.synchronize()
     assert out0.shape[0] == 0
     assert pa.device_error() == 0
+
+
+def test_prefill_output_16_byte_aligned(oracle):
+    """An output buffer that is 16- but not 32-byte aligned takes the 16-byte store path of the epilogue."""
+    rng = np.random.default_rng(41)
+    w = W.prefill_workload(256, [100, 37], 8, 2, 128, 256, rng=rng)
+    dw = DevicePrefill(w)
+    pa.store_kvcache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping)
+    T = dw.q.shape[0]
+    buf = torch.zeros(T * 8 * 128 + 8, dtype=torch.bfloat16, device="cuda")
+    out = buf[8:].view(T, 8, 128)                        # 16-byte offset from a 256-byte aligned allocation
+    assert out.data_ptr() % 32 == 16
+    pa.prefill_varlen(dw.q, dw.k_cache, dw.v_cache, dw.cu_seqlens_q, dw.cu_seqlens_k, w.max_seqlen_q,
+                      w.max_seqlen_k, dw.block_tables, w.scale, True, out=out)
+    ref_out = pa.prefill_varlen(dw.q, dw.k_cache, dw.v_cache, dw.cu_seqlens_q, dw.cu_seqlens_k, w.max_seqlen_q,
+                                w.max_seqlen_k, dw.block_tables, w.scale, True)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
+    assert not buf[:8].view(torch.int16).any()          # nothing written before the view
+    oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
+    _, ref = oracle.prefill_varlen(w.q, w.k_cache, w.v_cache, w.cu_seqlens_q, w.cu_seqlens_k, w.block_tables,
+                                   w.scale, True, want_f64=True)
+    assert_attention_close(out, ref, what="prefill, 16-byte aligned out")
+    assert pa.device_error() == 0
