@@ -8,7 +8,8 @@
  *   pa_rotary_store_kvcache
  *                      rotary embedding of q and k fused with that scatter
  *   pa_decode          one query token per sequence against its cached keys
- *                      (GQA; long contexts split across CTAs + a merge pass)
+ *                      (GQA; long contexts split across CTAs and merged by
+ *                      the last CTA of each sequence and kv head)
  *   pa_decode_partial, pa_merge_partials
  *                      the same split across GPUs: per-device partials,
  *                      combined after an all-gather
@@ -180,7 +181,7 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int3
  * g = h / (num_heads / num_kv_heads), K_j = k_cache[block_tables[b][j/bs]][j%bs][g]:
  *   out[b][h] = sum_{j<L} softmax_j(scale * <q[b][h], K_j>) * V_j
  * L == 0 gives out[b][h] = 0.  The newest token (position L-1) must already
- * be in the cache (call pa_store_kvcache first).
+ * be in the cache (call pa_store_kvcache first, or use pa_store_decode).
  *
  * q, out:         [num_seqs, num_heads, head_dim] bf16 (dense).
  * block_tables:   [num_seqs, max_blocks_per_seq] int32; entries past
@@ -190,7 +191,9 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int3
  *                 multiple of 64 (a value >= max_context_len disables the
  *                 split).  Sequences longer than one chunk are processed by
  *                 several CTAs whose partial (max, sum, weighted V) results
- *                 are merged by a second kernel.
+ *                 are merged by the last of them to finish (through device
+ *                 counters the library keeps and resets itself); above
+ *                 16384 sequences x kv heads a second kernel merges them.
  * workspace:      device buffer of at least pa_decode_workspace_size(...)
  *                 bytes (may be NULL when that size is 0); fully written
  *                 before it is read, so its contents need no initialisation.
