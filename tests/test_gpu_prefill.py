@@ -51,6 +51,71 @@ def test_prefill_small_shapes(oracle, prefix, sfx, hq, hkv, d, bs, causal):
     assert_attention_close(out, ref, what=f"prefill prefix={prefix} sfx={sfx} G={hq // hkv} D={d} bs={bs}")
 
 
+def lone_tiles(w, causal=True):
+    """Lone query tiles that see two key tiles or more, as (sequence, key tiles,
+    rows that see no key past the first key tile).  The kernel pairs a
+    sequence's 128-row query tiles (G heads x 128/G positions) into work items;
+    with an odd count the sequence's last tile runs alone."""
+    G = w.num_heads // w.num_kv_heads
+    qp = 128 // G
+    out = []
+    for b in range(w.num_seqs):
+        lq = int(w.cu_seqlens_q[b + 1] - w.cu_seqlens_q[b])
+        lk = int(w.cu_seqlens_k[b + 1] - w.cu_seqlens_k[b])
+        ntq = -(-lq // qp)
+        if ntq % 2 == 0:
+            continue
+        qt = ntq - 1
+        pos = [lk - lq + i for i in range(qt * qp, lq)]
+        nkeys = min(lk, pos[-1] + 1) if causal else lk
+        nt = -(-nkeys // 128)
+        if nt >= 2:
+            out.append((b, nt, sum(1 for p_ in pos if causal and p_ < 128)))
+    return out
+
+
+LONE_CASES = [
+    # prefix, suffixes, hq, hkv, d, bs, causal: every case has a lone query tile over two key tiles or more
+    (96, [50], 4, 2, 128, 32, True),                # 2 key tiles; rows at positions < 128 see none of tile 1
+    (96, [50, 30, 64], 8, 4, 64, 16, True),         # D 64; one lone tile over a single key tile
+    (0, [150, 130, 190], 2, 1, 128, 256, True),     # no prefix, lone third query tile
+    (512, [200, 150, 64], 16, 8, 128, 256, True),   # an even and an odd number of key tiles
+    (112, [100], 8, 8, 128, 16, True),              # G 1: 128 positions per tile
+    (112, [30, 90], 16, 4, 128, 16, True),          # G 4
+    (112, [40], 16, 2, 64, 16, True),               # G 8
+    (32, [150], 4, 2, 128, 16, False),              # non-causal
+    (1024, [64, 192, 320], 16, 8, 128, 256, True),  # 9 to 11 key tiles
+]
+
+
+@pytest.mark.parametrize("prefix,sfx,hq,hkv,d,bs,causal", LONE_CASES)
+def test_prefill_lone_query_tiles(oracle, prefix, sfx, hq, hkv, d, bs, causal):
+    rng = np.random.default_rng(7 * prefix + sum(sfx) + hq + d + bs)
+    w = W.prefill_workload(prefix, np.array(sfx, np.int32), hq, hkv, d, bs, rng=rng, causal=causal)
+    lone = lone_tiles(w, causal)
+    assert lone, "the case must contain a lone query tile over two key tiles or more"
+    out = store_and_prefill(DevicePrefill(w))
+    ref = oracle_prefill(oracle, w)
+    assert_attention_close(out, ref, what=f"lone-tile prefill prefix={prefix} sfx={sfx} G={hq // hkv} D={d} "
+                                          f"causal={causal} lone={lone}")
+
+
+def test_prefill_lone_cases_cover_the_edges():
+    """The lone-tile cases include rows that see no key past the first key tile, even and odd key-tile counts,
+    and every GQA group size the kernel instantiates."""
+    unseen, even, odd, groups = 0, 0, 0, set()
+    for prefix, sfx, hq, hkv, d, bs, causal in LONE_CASES:
+        w = W.prefill_workload(prefix, np.array(sfx, np.int32), hq, hkv, d, bs, rng=np.random.default_rng(0),
+                               causal=causal)
+        for _, nt, rows in lone_tiles(w, causal):
+            unseen += rows
+            even += nt % 2 == 0
+            odd += nt % 2 == 1
+        groups.add(hq // hkv)
+    assert unseen > 0 and even > 0 and odd > 0
+    assert groups == {1, 2, 4, 8}
+
+
 def test_prefill_prefix_workload_full_size_sampled(oracle):
     """The 32-sequence prefix-cached workload at full size; the oracle checks every 5th query token plus the
     first and last token of every sequence (all heads)."""
