@@ -22,9 +22,10 @@
 //              exponentials on the FMA pipe), writes P as bf16 pairs over the
 //              first half of its own S columns, rescales its O row in TMEM when
 //              the running max grows, and does the epilogue.
-//   warp 8     TMA producer: takes the next item, publishes it to the other
-//              warps through a shared-memory queue, loads its two Q tiles,
-//              then its K and V tiles in rings (K one tile ahead).
+//   warp 8     TMA producer: takes the next item, decodes it and publishes
+//              the decoded item to the other warps through a shared-memory
+//              queue, loads its two Q tiles, then its K and V tiles in rings
+//              (K one tile ahead).
 //   warps 10-11 idle (they complete the third warpgroup, whose registers
 //              the softmax warpgroups borrow through setmaxnreg).
 //   warp 9     TMEM allocator and single-thread MMA issuer, in the order
@@ -106,7 +107,9 @@ struct PrefillSmem {
   static constexpr int kNumBars = 1 + 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1 + 2 * kWorkQ;
   static constexpr size_t tmem_slot_off = bar_off + kNumBars * 8;
   static constexpr size_t queue_off = tmem_slot_off + 16;
-  static constexpr size_t bytes = queue_off + kWorkQ * 4;
+  static constexpr size_t kItemBytes = 64;              // one decoded work item (struct Item)
+  static constexpr size_t items_off = queue_off + kWorkQ * 4;
+  static constexpr size_t bytes = items_off + kWorkQ * kItemBytes;
   static_assert(bytes <= 232448, "shared memory budget (227 KB per CTA)");
 };
 
@@ -252,7 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = o_done + 2;
   uint64_t* work_full = mma_done + 1;        // [kWorkQ]: queue entry written (producer)
   uint64_t* work_empty = work_full + Smem::kWorkQ;   // [kWorkQ]: entry read by the MMA thread and 8 softmax warps
+  // queue entries: the item number (-1: no more work) and the item as the
+  // producer decoded it, so that the other roles do not decode it again
   int32_t* work_queue = reinterpret_cast<int32_t*>(smem + Smem::queue_off);
+  Item* work_items = reinterpret_cast<Item*>(smem + Smem::items_off);
+  static_assert(sizeof(Item) <= Smem::kItemBytes && Smem::items_off % alignof(Item) == 0, "work item slot");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Smem::tmem_slot_off);
   constexpr int kWorkQ = Smem::kWorkQ;
 
@@ -316,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = n % kWorkQ;
         if (!(ok = mbar_wait(&work_empty[q], ((n / kWorkQ) & 1) ^ 1, p.err))) break;
         work_queue[q] = t < num_items ? t : -1;
+        if (t < num_items) work_items[q] = it;
         mbar_arrive(&work_full[q]);   // release: the entry is visible to waiters of this phase
         if (t >= num_items) break;
         const int32_t* bt = p.block_tables + static_cast<int64_t>(it.b) * p.max_blocks_per_seq;
@@ -410,9 +418,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = n % kWorkQ;
         if (!(ok = mbar_wait(&work_full[q], (n / kWorkQ) & 1, p.err))) break;
         const int t = work_queue[q];
+        Item it;
+        if (t >= 0) it = work_items[q];
         mbar_arrive(&work_empty[q]);
         if (t < 0) break;
-        const Item it = decode_item<QP>(t, num_seqs, num_kv_heads, p);
         const int ntA = it.ntA, ntB = it.ntB;
         if (!(ok = mbar_wait(q_full, nitems & 1, p.err))) break;
         ++nitems;
@@ -483,10 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q = n % kWorkQ;
       if (!(ok = mbar_wait_warp(&work_full[q], (n / kWorkQ) & 1, p.err))) break;
       const int t = work_queue[q];
+      Item it;
+      if (t >= 0) it = work_items[q];
       __syncwarp();
       if (lane == 0) mbar_arrive(&work_empty[q]);
       if (t < 0) break;
-      const Item it = decode_item<QP>(t, num_seqs, num_kv_heads, p);
       const int ntx = x == 0 ? it.ntA : it.ntB;
       if (ntx == 0) continue;
       const int full_keys = x == 0 ? it.fullA : it.fullB;
