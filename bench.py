@@ -389,18 +389,20 @@ def bench_prefill(args, dev, peaks):
     tflops = flops / (prefill_ms / 1e3) / 1e12
     # the SM clock under a sustained prefill load: back-to-back launches for about half a second (K/V of this
     # workload stay in L2, so this is a clock record, not the reported time)
-    n_sus = int(min(5000, max(50, 0.5 / (prefill_ms / 1e3))))
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clk:
-        s0.record()
-        for _ in range(n_sus):
-            prefill()
-        s1.record()
-        torch.cuda.synchronize(dev)
-    assert pa.device_error() == 0
-    sus_ms = s0.elapsed_time(s1) / n_sus
-    sustained = {"launches": n_sus, "ms": sus_ms, "tflops": flops / (sus_ms / 1e3) / 1e12,
-                 "note": "back to back, L2 warm", "clocks": clk.summary()}
+    sustained = None
+    if not args.no_prefill_clock:
+        n_sus = int(min(5000, max(50, 0.5 / (prefill_ms / 1e3))))
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(dev.index) as clk:
+            s0.record()
+            for _ in range(n_sus):
+                prefill()
+            s1.record()
+            torch.cuda.synchronize(dev)
+        assert pa.device_error() == 0
+        sus_ms = s0.elapsed_time(s1) / n_sus
+        sustained = {"launches": n_sus, "ms": sus_ms, "tflops": flops / (sus_ms / 1e3) / 1e12,
+                     "note": "back to back, L2 warm", "clocks": clk.summary()}
     store_bytes = 2 * 2 * int(w.cu_seqlens_q[-1]) * w.num_kv_heads * w.head_dim * 2 + 4 * int(w.cu_seqlens_q[-1])
     store_gbs = store_bytes / (store_ms / 1e3) / 1e9
     rot = bench_rotary_store(w, dev, q, nk, nv, kc, vc, slots, flush, reps)
@@ -679,6 +681,8 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-prefill-clock", action="store_true",
+                    help="skip the sustained prefill loop that records the SM clock under prefill load")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
