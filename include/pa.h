@@ -163,6 +163,19 @@ PA_API pa_status pa_rotary_store_kvcache(void* q_out, const void* q, int64_t q_r
 PA_API int32_t pa_decode_chunk_size(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int32_t block_size);
 
 /*
+ * pa_decode_chunk_size_for -- the same choice for a device with sm_count
+ * streaming multiprocessors, without querying any device (usable on a host
+ * with no GPU, e.g. to plan workspace sizes).  The choice aims at about four
+ * waves of two CTAs per SM: no split while num_seqs * num_kv_heads already
+ * reaches 8 * sm_count or max_context_len <= 512; otherwise the split count
+ * within one of that target whose chunks (whole 64-token tiles) overhang the
+ * longest context least, and at most ceil(max_context_len / 512) chunks.
+ * Returns -1 for invalid arguments.
+ */
+PA_API int32_t pa_decode_chunk_size_for(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len,
+                                        int32_t sm_count);
+
+/*
  * pa_decode_workspace_size -- bytes of workspace pa_decode needs for these
  * arguments (0 when no sequence is split).  kv_chunk_size as for pa_decode.
  * Returns 0 for invalid arguments as well; pa_decode then reports them.

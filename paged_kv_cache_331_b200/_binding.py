@@ -25,6 +25,7 @@ _PROTOS = {
     "pa_version": (_i32, []),
     "pa_store_kvcache": (ctypes.c_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pa_decode_chunk_size": (_i32, [_i32, _i32, _i32, _i32]),
+    "pa_decode_chunk_size_for": (_i32, [_i32, _i32, _i32, _i32]),
     "pa_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
     "pa_decode": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                  _i32, _vp, _sz, _vp]),
@@ -152,6 +153,10 @@ def rotary_store_kvcache(q, key, value, positions, cos_sin_cache, k_cache, v_cac
 
 def decode_chunk_size(num_seqs, num_kv_heads, max_context_len, block_size) -> int:
     return int(lib().pa_decode_chunk_size(num_seqs, num_kv_heads, max_context_len, block_size))
+
+
+def decode_chunk_size_for(num_seqs, num_kv_heads, max_context_len, sm_count) -> int:
+    return int(lib().pa_decode_chunk_size_for(num_seqs, num_kv_heads, max_context_len, sm_count))
 
 
 def decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, block_size,

@@ -247,6 +247,11 @@ int32_t pa_decode_chunk_size(int32_t num_seqs, int32_t num_kv_heads, int32_t max
   return decode_auto_chunk(num_seqs, num_kv_heads, max_context_len, current_device_info()->sm_count);
 }
 
+int32_t pa_decode_chunk_size_for(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int32_t sm_count) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || max_context_len < 0 || sm_count <= 0) return -1;
+  return decode_auto_chunk(num_seqs, num_kv_heads, max_context_len, sm_count);
+}
+
 static int32_t resolve_chunk(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int32_t kv_chunk_size) {
   if (kv_chunk_size == 0)
     return decode_auto_chunk(num_seqs, num_kv_heads, max_context_len, current_device_info()->sm_count);
