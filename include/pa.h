@@ -330,6 +330,12 @@ PA_API pa_status pa_merge_partials(void* out, const float* o_parts, const float*
  * cu_seqlens_q/k: [num_seqs+1] int32, non-decreasing.
  * max_seqlen_q/k: upper bounds of Lq and Lk over the batch.
  * block_tables:   as for pa_decode, entries past ceil(Lk/block_size) unread.
+ *
+ * Preconditions on device data that the kernel does not check: total_q and
+ * max_seqlen_q/k agree with cu_seqlens_q/k, and Lk <= max_blocks_per_seq *
+ * block_size.  A violation can read or write outside the caller's buffers.
+ * (pa_decode, by contrast, clamps each context length to max_context_len and
+ * to the table width.)
  */
 PA_API pa_status pa_prefill_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t total_q,
