@@ -82,6 +82,32 @@ def _dense(t: torch.Tensor, name: str) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
+def _same_device(ref: torch.Tensor, **tensors) -> None:
+    """Every tensor of one call lives on the device of ``ref``: a pointer into
+    another GPU's memory would reach a kernel that cannot read it."""
+    for name, t in tensors.items():
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, the call's other tensors on {ref.device}")
+
+
+def _shape(t: torch.Tensor, shape, name: str) -> None:
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _rows(t: torch.Tensor, n: int, name: str, dim: int) -> None:
+    """A per-sequence array (``dim`` dimensions) with at least one row per sequence; rows past n are not read."""
+    if t.dim() != dim or t.shape[0] < n:
+        raise ValueError(f"{name} must be {dim}-D with at least {n} rows, got shape {tuple(t.shape)}")
+
+
+def _caches(k_cache: torch.Tensor, v_cache: torch.Tensor, head_dim=None) -> None:
+    if k_cache.dim() != 4 or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache and v_cache must both be [num_blocks, block_size, num_kv_heads, head_dim]")
+    if head_dim is not None and k_cache.shape[3] != head_dim:
+        raise ValueError(f"head_dim of the cache ({k_cache.shape[3]}) and of q ({head_dim}) differ")
+
+
 def _stream(t: torch.Tensor, stream) -> int:
     s = stream if stream is not None else torch.cuda.current_stream(t.device)
     return s.cuda_stream
@@ -93,6 +119,10 @@ def store_kvcache(key, value, k_cache, v_cache, slot_mapping, stream=None) -> No
         _cuda(t, n, torch.bfloat16)
     _cuda(slot_mapping, "slot_mapping", torch.int32)
     _dense(k_cache, "k_cache"); _dense(v_cache, "v_cache"); _dense(slot_mapping, "slot_mapping")
+    _caches(k_cache, v_cache)
+    _same_device(k_cache, key=key, value=value, v_cache=v_cache, slot_mapping=slot_mapping)
+    if slot_mapping.dim() != 1:
+        raise ValueError("slot_mapping must be [N]")
     nb, bs, hkv, d = k_cache.shape
     n = slot_mapping.shape[0]
     for name, t in (("key", key), ("value", value)):
@@ -127,7 +157,10 @@ def rotary_store_kvcache(q, key, value, positions, cos_sin_cache, k_cache, v_cac
     for n, t in (("k_cache", k_cache), ("v_cache", v_cache), ("positions", positions), ("slot_mapping", slot_mapping),
                  ("cos_sin_cache", cos_sin_cache)):
         _dense(t, n)
+    _caches(k_cache, v_cache)
     nb, bs, hkv, d = k_cache.shape
+    if q.dim() != 3:
+        raise ValueError("q must be [N, Hq, D]")
     n, hq = q.shape[0], q.shape[1]
     if tuple(q.shape[1:]) != (hq, d) or q.stride(-1) != 1 or q.stride(-2) != d:
         raise ValueError(f"q must be [N, Hq, {d}] with dense rows")
@@ -142,6 +175,9 @@ def rotary_store_kvcache(q, key, value, positions, cos_sin_cache, k_cache, v_cac
         out = torch.empty(n, hq, d, dtype=torch.bfloat16, device=q.device)
     _cuda(out, "out", torch.bfloat16)
     _dense(out, "out")
+    _shape(out, (n, hq, d), "out")
+    _same_device(k_cache, q=q, key=key, value=value, positions=positions, cos_sin_cache=cos_sin_cache,
+                 v_cache=v_cache, slot_mapping=slot_mapping, out=out)
     with torch.cuda.device(k_cache.device):
         _check(lib().pa_rotary_store_kvcache(out.data_ptr(), q.data_ptr(), q.stride(0), key.data_ptr(),
                                              value.data_ptr(), key.stride(0), value.stride(0), positions.data_ptr(),
@@ -173,16 +209,19 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len, sca
     _cuda(block_tables, "block_tables", torch.int32); _dense(block_tables, "block_tables")
     _cuda(context_lens, "context_lens", torch.int32); _dense(context_lens, "context_lens")
     B, hq, d = q.shape
-    nb, bs, hkv, d2 = k_cache.shape
-    if d2 != d:
-        raise ValueError("head_dim of q and the cache differ")
+    _caches(k_cache, v_cache, d)
+    nb, bs, hkv, _ = k_cache.shape
+    _rows(block_tables, B, "block_tables", 2)
+    _rows(context_lens, B, "context_lens", 1)
     if out is None:
         out = torch.empty_like(q)
     else:
-        _cuda(out, "out", torch.bfloat16); _dense(out, "out")
+        _cuda(out, "out", torch.bfloat16); _dense(out, "out"); _shape(out, q.shape, "out")
     need = decode_workspace_size(B, hq, hkv, d, int(max_context_len), bs, kv_chunk_size)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _same_device(q, k_cache=k_cache, v_cache=v_cache, block_tables=block_tables, context_lens=context_lens, out=out,
+                 workspace=workspace)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
     with torch.cuda.device(q.device):
@@ -204,15 +243,23 @@ def store_decode(q, key, value, slot_mapping, k_cache, v_cache, block_tables, co
         _cuda(t, n, torch.int32)
         _dense(t, n)
     B, hq, d = q.shape
+    _caches(k_cache, v_cache, d)
     nb, bs, hkv, _ = k_cache.shape
     for name, t in (("key", key), ("value", value)):
         if t.shape[0] != B or tuple(t.shape[1:]) != (hkv, d) or t.stride(-1) != 1 or t.stride(-2) != d:
             raise ValueError(f"{name} must be [B, {hkv}, {d}] with dense rows")
+    _rows(slot_mapping, B, "slot_mapping", 1)
+    _rows(block_tables, B, "block_tables", 2)
+    _rows(context_lens, B, "context_lens", 1)
     if out is None:
         out = torch.empty_like(q)
+    else:
+        _cuda(out, "out", torch.bfloat16); _dense(out, "out"); _shape(out, q.shape, "out")
     need = decode_workspace_size(B, hq, hkv, d, int(max_context_len), bs, kv_chunk_size)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _same_device(q, key=key, value=value, slot_mapping=slot_mapping, k_cache=k_cache, v_cache=v_cache,
+                 block_tables=block_tables, context_lens=context_lens, out=out, workspace=workspace)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
     with torch.cuda.device(q.device):
@@ -235,7 +282,10 @@ def decode_partial(q, k_cache, v_cache, block_tables, context_lens, max_context_
     _dense(block_tables, "block_tables")
     _dense(context_lens, "context_lens")
     B, hq, d = q.shape
+    _caches(k_cache, v_cache, d)
     nb, bs, hkv, _ = k_cache.shape
+    _rows(block_tables, B, "block_tables", 2)
+    _rows(context_lens, B, "context_lens", 1)
     if o_part is None:
         o_part = torch.empty(B, hq, d, dtype=torch.float32, device=q.device)
     if lse_part is None:
@@ -243,9 +293,13 @@ def decode_partial(q, k_cache, v_cache, block_tables, context_lens, max_context_
     for n, t in (("o_part", o_part), ("lse_part", lse_part)):
         _cuda(t, n, torch.float32)
         _dense(t, n)
+    _shape(o_part, (B, hq, d), "o_part")
+    _shape(lse_part, (B, hq), "lse_part")
     need = decode_workspace_size(B, hq, hkv, d, int(max_context_len), bs, kv_chunk_size)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _same_device(q, k_cache=k_cache, v_cache=v_cache, block_tables=block_tables, context_lens=context_lens,
+                 o_part=o_part, lse_part=lse_part, workspace=workspace)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
     with torch.cuda.device(q.device):
@@ -263,6 +317,8 @@ def merge_partials(o_parts, lse_parts, *, out=None, stream=None):
     _cuda(lse_parts, "lse_parts", torch.float32)
     _dense(o_parts, "o_parts")
     _dense(lse_parts, "lse_parts")
+    if o_parts.dim() != 4:
+        raise ValueError("o_parts must be [R, B, Hq, D]")
     R, B, hq, d = o_parts.shape
     if tuple(lse_parts.shape) != (R, B, hq):
         raise ValueError("lse_parts must be [R, B, Hq]")
@@ -270,6 +326,8 @@ def merge_partials(o_parts, lse_parts, *, out=None, stream=None):
         out = torch.empty(B, hq, d, dtype=torch.bfloat16, device=o_parts.device)
     _cuda(out, "out", torch.bfloat16)
     _dense(out, "out")
+    _shape(out, (B, hq, d), "out")
+    _same_device(o_parts, lse_parts=lse_parts, out=out)
     with torch.cuda.device(o_parts.device):
         _check(lib().pa_merge_partials(out.data_ptr(), o_parts.data_ptr(), lse_parts.data_ptr(), R, B * hq, d,
                                        _stream(o_parts, stream)), "pa_merge_partials")
@@ -287,7 +345,12 @@ def decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, max_context_
     _cuda(block_tables, "block_tables", torch.int32); _dense(block_tables, "block_tables")
     _cuda(context_lens, "context_lens", torch.int32); _dense(context_lens, "context_lens")
     B, hq, d = q.shape
+    _caches(k_cache, v_cache, d)
     nb, bs, hkv, _ = k_cache.shape
+    _rows(block_tables, B, "block_tables", 2)
+    _rows(context_lens, B, "context_lens", 1)
+    _shape(out, q.shape, "out")
+    _same_device(q, k_cache=k_cache, v_cache=v_cache, block_tables=block_tables, context_lens=context_lens, out=out)
     with torch.cuda.device(q.device):
         _check(lib().pa_decode_noalloc(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
                                        block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
@@ -304,16 +367,24 @@ def prefill_varlen(q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q
     for n, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k), ("block_tables", block_tables)):
         _cuda(t, n, torch.int32); _dense(t, n)
     total_q, hq, d = q.shape
+    _caches(k_cache, v_cache, d)
     nb, bs, hkv, _ = k_cache.shape
+    if cu_seqlens_q.dim() != 1 or cu_seqlens_q.shape[0] < 1:
+        raise ValueError("cu_seqlens_q must be [num_seqs + 1]")
+    num_seqs = cu_seqlens_q.shape[0] - 1
+    _rows(cu_seqlens_k, num_seqs + 1, "cu_seqlens_k", 1)
+    _rows(block_tables, num_seqs, "block_tables", 2)
     if out is None:
         out = torch.empty_like(q)
     else:
-        _cuda(out, "out", torch.bfloat16); _dense(out, "out")
+        _cuda(out, "out", torch.bfloat16); _dense(out, "out"); _shape(out, q.shape, "out")
+    _same_device(q, k_cache=k_cache, v_cache=v_cache, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+                 block_tables=block_tables, out=out)
     with torch.cuda.device(q.device):
         _check(lib().pa_prefill_varlen(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
                                        cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), total_q, int(max_seqlen_q),
                                        int(max_seqlen_k), block_tables.data_ptr(), block_tables.shape[1],
-                                       cu_seqlens_q.shape[0] - 1, hq, hkv, d, bs, nb, float(scale), int(bool(causal)),
+                                       num_seqs, hq, hkv, d, bs, nb, float(scale), int(bool(causal)),
                                        _stream(q, stream)), "pa_prefill_varlen")
     return out
 
