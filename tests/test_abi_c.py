@@ -1,7 +1,7 @@
 """The C ABI from C (CPU only): a plain C client (tests/c_abi_client.c) is compiled
 against include/*.h, linked to libpagedattn.so and run; its view of the host-side
 entry points must agree with the Python binding, the xxhash package and the
-block-manager oracle."""
+block-manager oracle.  The same client also compiles as C++."""
 import subprocess
 from pathlib import Path
 
@@ -26,6 +26,18 @@ def client_output(tmp_path_factory):
     return {line.split()[0]: line.split()[1:] for line in r.stdout.splitlines() if line.strip()
             if not line.startswith("status ")} | \
         {"status": [line.split()[1:] for line in r.stdout.splitlines() if line.startswith("status ")]}
+
+
+def test_headers_compile_as_cxx(tmp_path):
+    """The same client compiled as C++ (the headers' extern "C" guards) links and prints the same lines."""
+    from paged_kv_cache_331_b200 import build as B
+    B.build()
+    exe = tmp_path / "client_cxx"
+    subprocess.run(["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-x", "c++", f"-I{ROOT / 'include'}",
+                    str(ROOT / "tests" / "c_abi_client.c"), f"-L{PKG}", "-lpagedattn", f"-Wl,-rpath,{PKG}",
+                    "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
+    assert out.startswith("version ") and "unknown_sequence 1" in out
 
 
 def test_status_and_version(client_output):
