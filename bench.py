@@ -178,14 +178,14 @@ def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl != "ours":
+        return world, rank, local      # the reference arm runs on rank 0 alone and takes no collective step
     if world > 1:
         import datetime
         import torch.distributed as dist
-        backend = "nccl" if args.impl == "ours" else "gloo"
-        if backend == "nccl":
-            torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
-    elif args.impl == "ours":
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -633,13 +633,13 @@ def run_reference(args, world, rank):
     from paged_kv_cache_331_b200 import workloads as W
     orc = O.get()
     w = W.qwen3_decode()
-    # calibrate: sequences per step so that warmup + steps end within about two minutes
+    # calibrate: sequences per step so that warmup + steps end within about --reference-seconds
     one = W.decode_workload(w.context_lens[:1], w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
                             rng=np.random.default_rng(0))
     t = time.perf_counter()
     orc.decode(one.q, one.k_cache, one.v_cache, one.block_tables, one.context_lens, one.scale)
     t1 = max(time.perf_counter() - t, 1e-4) * max(1.0, 2112.0 / float(one.context_lens[0]))
-    per_step_budget = 120.0 / max(1, args.steps + args.warmup)
+    per_step_budget = args.reference_seconds / max(1, args.steps + args.warmup)
     nseq = int(max(1, min(w.num_seqs, per_step_budget / t1)))
     sub = slice(0, nseq)
     kc, vc = w.k_cache.copy(), w.v_cache.copy()
@@ -681,6 +681,8 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--reference-seconds", type=float, default=120.0,
+                    help="--impl reference: about how long the oracle's warm-up and timed steps take together")
     ap.add_argument("--no-prefill-clock", action="store_true",
                     help="skip the sustained prefill loop that records the SM clock under prefill load")
     args = ap.parse_args()
@@ -693,7 +695,7 @@ def main():
         else:
             run_ours(args, world, rank, local)
     finally:
-        if world > 1:
+        if world > 1 and args.impl == "ours":
             import torch.distributed as dist
             dist.barrier()
             dist.destroy_process_group()
