@@ -265,6 +265,10 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache
  * error code 5.  key/value rows must be 16-byte aligned with strides that are
  * multiples of 8 elements (PA_ERR_UNSUPPORTED otherwise).  Every other
  * argument, the workspace rule and the errors are pa_decode's.
+ * Precondition the kernel does not check: the block-table entry that covers
+ * position context_lens[b]-1 is a valid block id (< num_blocks); the row is
+ * written at the slot that entry names.  (pa_store_kvcache skips a slot
+ * outside the cache instead.)
  */
 PA_API pa_status pa_store_decode(void* out, const void* q, const void* key, const void* value, int64_t key_row_stride,
                           int64_t value_row_stride, const int32_t* slot_mapping, void* k_cache, void* v_cache,
