@@ -233,8 +233,11 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, max_context_len, sca
 
 
 def store_decode(q, key, value, slot_mapping, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, *,
-                 out=None, workspace=None, kv_chunk_size=0, stream=None):
-    """pa_store_decode: store each sequence's new K/V row (slot of position L-1, or -1) and decode, one launch."""
+                 out=None, workspace=None, kv_chunk_size=0, stream=None, validate=False):
+    """pa_store_decode: store each sequence's new K/V row (slot of position L-1, or -1) and decode, one launch.
+
+    ``validate=True`` first checks on the host (a synchronising copy) that every slot is the one its block table
+    names for the newest position, through a valid block id: the kernel takes that on trust."""
     for n, t in (("q", q), ("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache)):
         _cuda(t, n, torch.bfloat16)
     for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
@@ -260,6 +263,9 @@ def store_decode(q, key, value, slot_mapping, k_cache, v_cache, block_tables, co
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     _same_device(q, key=key, value=value, slot_mapping=slot_mapping, k_cache=k_cache, v_cache=v_cache,
                  block_tables=block_tables, context_lens=context_lens, out=out, workspace=workspace)
+    if validate:
+        from .metadata import check_store_decode_metadata
+        check_store_decode_metadata(slot_mapping[:B], block_tables[:B], context_lens[:B], int(max_context_len), bs, nb)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
     with torch.cuda.device(q.device):
@@ -360,8 +366,11 @@ def decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, max_context_
 
 
 def prefill_varlen(q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, block_tables, scale,
-                   causal=True, *, out=None, stream=None):
-    """Varlen prefill over the paged cache: q [total_q, Hq, D] -> out [total_q, Hq, D]."""
+                   causal=True, *, out=None, stream=None, validate=False):
+    """Varlen prefill over the paged cache: q [total_q, Hq, D] -> out [total_q, Hq, D].
+
+    ``validate=True`` first checks on the host (a synchronising copy) what the kernel takes on trust: the
+    cu_seqlens agree with total_q, max_seqlen_q/k and the block tables, whose entries are valid block ids."""
     for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _cuda(t, n, torch.bfloat16); _dense(t, n)
     for n, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k), ("block_tables", block_tables)):
@@ -380,6 +389,10 @@ def prefill_varlen(q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q
         _cuda(out, "out", torch.bfloat16); _dense(out, "out"); _shape(out, q.shape, "out")
     _same_device(q, k_cache=k_cache, v_cache=v_cache, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
                  block_tables=block_tables, out=out)
+    if validate:
+        from .metadata import check_prefill_metadata
+        check_prefill_metadata(cu_seqlens_q, cu_seqlens_k[:num_seqs + 1], total_q, int(max_seqlen_q),
+                               int(max_seqlen_k), block_tables, bs, nb)
     with torch.cuda.device(q.device):
         _check(lib().pa_prefill_varlen(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
                                        cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), total_q, int(max_seqlen_q),
