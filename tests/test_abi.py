@@ -87,3 +87,55 @@ def test_workspace_size_arithmetic(libpa):
     assert n == (rows * D * 4 + 255) // 256 * 256 + rows * 2 * 4
     assert libpa.pa_decode_workspace_size(B, H, Hkv, D, 256, 16, 256) == 0     # one chunk: no workspace
     assert libpa.pa_decode_workspace_size(B, H, Hkv, D, 1000, 16, 100) == 0    # invalid chunk -> 0
+
+
+def test_more_rejections_before_any_launch(libpa):
+    """Each call breaks one rule of its entry point and is refused with that rule's status, before any launch:
+    1 = PA_ERR_INVALID_ARG, 2 = PA_ERR_UNSUPPORTED."""
+    L, null = libpa, None
+    mis = 0x1003                                             # a misaligned (never dereferenced) address
+    # store_kvcache: a non-positive size, a row too long for the kernel
+    assert L.pa_store_kvcache(null, null, 64, 64, null, null, null, 1, 0, 64, 16, 4, null) == 1
+    assert L.pa_store_kvcache(null, null, 1 << 21, 1 << 21, null, null, null, 1, 2048, 1024, 16, 4, null) == 2
+    # rotary table: null table, odd head_dim, base <= 1
+    assert L.pa_rotary_cos_sin_cache(null, 16, 64, 1e4, null) == 1
+    assert L.pa_rotary_cos_sin_cache(mis, 16, 63, 1e4, null) == 1
+    assert L.pa_rotary_cos_sin_cache(mis, 16, 64, 1.0, null) == 1
+
+    # rotary store: head_dim, head count, short q stride, null pointers, misaligned pointers
+    def rot(d=64, hq=4, hkv=2, q_stride=None, ptr=null, n=3):
+        qs = q_stride if q_stride is not None else hq * d
+        return L.pa_rotary_store_kvcache(ptr, ptr, qs, ptr, ptr, hkv * d, hkv * d, ptr, ptr, 16, ptr, ptr, ptr, n,
+                                         hq, hkv, d, 16, 4, null)
+    assert rot(d=96) == 2
+    assert rot(hq=8192) == 2
+    assert rot(q_stride=10) == 1
+    assert rot() == 1                                        # null pointers
+    assert rot(ptr=mis) == 2                                 # 16-byte alignment
+    assert rot(n=0) == 0                                     # nothing to do
+
+    # decode: scale, negative context bound, table width
+    dargs = lambda scale=0.125, maxL=100, mb=4: (null, null, null, null, null, mb, null, maxL, 2, 4, 2, 64, 16, 8,
+                                                 scale, 0, null, 0, null)
+    assert L.pa_decode(*dargs(scale=0.0)) == 1
+    assert L.pa_decode(*dargs(scale=float("nan"))) == 1
+    assert L.pa_decode(*dargs(maxL=-1)) == 1
+    assert L.pa_decode(*dargs(mb=0)) == 1
+
+    # prefill: negative counts, scale, table width
+    pargs = lambda ns=4, tq=10, scale=0.125, mb=4: (null, null, null, null, null, null, tq, 8, 8, null, mb, ns, 4, 2,
+                                                    64, 16, 8, scale, 1, null)
+    assert L.pa_prefill_varlen(*pargs(ns=-1)) == 1
+    assert L.pa_prefill_varlen(*pargs(tq=-1)) == 1
+    assert L.pa_prefill_varlen(*pargs(scale=-1.0)) == 1
+    assert L.pa_prefill_varlen(*pargs(mb=0)) == 1
+    assert L.pa_prefill_varlen(*pargs(tq=0)) == 0            # no query rows: nothing to do
+
+    # merge_partials: no partials, head_dim, null and misaligned pointers
+    assert L.pa_merge_partials(null, null, null, 0, 4, 64, null) == 1
+    assert L.pa_merge_partials(null, null, null, 2, 4, 96, null) == 2
+    assert L.pa_merge_partials(null, null, null, 2, 4, 64, null) == 1
+    assert L.pa_merge_partials(mis, mis, mis, 2, 4, 64, null) == 1
+    assert L.pa_merge_partials(null, null, null, 2, 0, 64, null) == 0
+
+    assert L.pa_status_string(99) == b"PA_ERR_UNKNOWN"
