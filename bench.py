@@ -3,16 +3,24 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one decode step of the Qwen3-0.6B-shaped layer (64 sequences,
-context U[128,4096], 16 q / 8 kv heads, head_dim 128, block_size 256):
-store_kvcache of the 64 new K/V rows, then paged GQA decode with split-KV and
-its merge pass.  Inputs are resident in HBM when the timed region starts;
-the KV working set (~0.55 GB) is larger than L2, so repeated steps read HBM.
-The headline value is decode KV bytes per second over all ranks.  The same
-JSON line carries the prefix-cached varlen prefill leg (32 sequences behind a
-shared 1024-token prefix) in TFLOP/s, the end-to-end number through host
-buffers, the roofline of the dominant kernel, and the oracle timed on the
-host cores.
+A step is one decode step of the large-batch layer (256 sequences, context
+U[100,1024] prompt + U[1,1024] generated, 32 q / 8 kv heads, head_dim 128,
+block_size 256): store_kvcache of the 256 new K/V rows, then paged GQA decode
+of every sequence, in one pa_store_decode launch.  It is the largest decode
+workload that fits one GPU (~1.13 GB of KV per step, far more than L2), so
+repeated steps read HBM; inputs are resident in HBM when the timed region
+starts.  The headline value is decode KV bytes per second over all ranks.
+
+The same JSON line carries, each with its own roofline:
+  decode_workloads   the other decode workloads timed on their own: the tiny
+                     4-sequence case (latency), the Qwen3-0.6B-shaped layer
+                     (64 sequences) and the long-context split-KV case
+                     (8 x 32768 + 1)
+  store_256_rows     the headline step's 256-row store on its own (us, GB/s)
+  prefill            the prefix-cached varlen prefill (32 sequences behind a
+                     shared 1024-token prefix) in TFLOP/s, with its suffix store
+  e2e                the headline step through host buffers (copies included)
+  cpu_baseline       the oracle timed on the host cores
 
 Under torchrun every rank runs its own independent batch (no collective on
 the data path); the timed region is bracketed by barriers and the reported
@@ -151,24 +159,32 @@ class ClockSampler:
         if self._nvml is not None:
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
+            t0 = time.perf_counter()       # running before the timed region starts: wait for its first samples
+            while len(self.samples) < 2 and self.err is None and time.perf_counter() - t0 < 2.0:
+                time.sleep(0.0005)
         return self
+
+    def mark(self):
+        """Index of the next sample (to tell which samples fall inside a timed region)."""
+        return len(self.samples)
 
     def __exit__(self, *exc):
         self._stop.set()
         if self._thread:
             self._thread.join()
 
-    def summary(self):
-        if not self.samples:
+    def summary(self, lo=0, hi=None):
+        samples = self.samples[lo:hi]
+        if not samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
                     "note": self.err or "no samples"}
-        mhz = [s[0] for s in self.samples]
+        mhz = [s[0] for s in samples]
         bits = 0
-        for s in self.samples:
+        for s in samples:
             bits |= s[2]
         reasons = sorted(name for bit, name in self.REASONS.items() if bits & bit)
         return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(self.samples), "power_w_max": round(max(s[1] for s in self.samples), 1)}
+                "samples": len(samples), "power_w_max": round(max(s[1] for s in samples), 1)}
 
 
 # ---------------------------------------------------------------------------------------- distributed --
@@ -236,105 +252,256 @@ def pinned(a, kind):
     return t.pin_memory()
 
 
+def decode_config(w, context_desc):
+    """The workload as both arms name it: shapes, context distribution, pool and the KV bytes of one step."""
+    kv, _ = decode_algorithmic_bytes(w)
+    return {"workload": w.name, "num_seqs": w.num_seqs, "context_lens": context_desc, "num_heads": w.num_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+            "pool_blocks": w.num_blocks, "kv_bytes_per_step": kv,
+            "l2": (f"inputs larger than L2: {kv / 1e6:.0f} MB KV per step vs 126 MB L2" if kv > 126e6 else
+                   f"{kv / 1e6:.2f} MB of KV: L2-resident between steps (a latency case)")}
+
+
+HEADLINE = ("large_batch_decode", "U[100,1024] prompt + U[1,1024] generated")
+DECODE_LEGS = {   # the other decode workloads, each timed as its own leg of the same run
+    "tiny_decode": "{1,17,256,300}",
+    "qwen3_decode": "U[128,4096]",
+    "long_context_decode": "8 x 32768 + 1 x 1",
+}
+
+
+class DecodeOnDevice:
+    """A decode workload resident on the GPU, with its output, workspace and chunk choice."""
+
+    def __init__(self, w, dev, kv_chunk_size=0):
+        import torch
+        import paged_kv_cache_331_b200 as pa
+        self.w = w
+        self.q, self.kc, self.vc = to_dev(w.q, "bf16", dev), to_dev(w.k_cache, "bf16", dev), to_dev(w.v_cache, "bf16", dev)
+        self.nk, self.nv = to_dev(w.new_k, "bf16", dev), to_dev(w.new_v, "bf16", dev)
+        self.slots, self.bt = to_dev(w.slot_mapping, "i32", dev), to_dev(w.block_tables, "i32", dev)
+        self.cl = to_dev(w.context_lens, "i32", dev)
+        self.out = torch.empty_like(self.q)
+        self.maxL = w.max_context_len
+        self.chunk_arg = kv_chunk_size
+        self.ws_bytes = pa.decode_workspace_size(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, self.maxL,
+                                                 w.block_size, kv_chunk_size)
+        self.ws = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.chunk = (pa.decode_chunk_size(w.num_seqs, w.num_kv_heads, self.maxL, w.block_size)
+                      if kv_chunk_size == 0 else kv_chunk_size)
+        nchunks = -(-self.maxL // self.chunk) if self.maxL else 1
+        # one launch per step, plus the separate merge kernel above 16384 split sequences x kv heads
+        self.launches_per_step = 1 + int(nchunks > 1 and w.num_seqs * w.num_kv_heads > 16384)
+
+    def step(self):
+        """One decode step: the new rows stored and every sequence decoded, in one pa_store_decode launch."""
+        import paged_kv_cache_331_b200 as pa
+        pa.store_decode(self.q, self.nk, self.nv, self.slots, self.kc, self.vc, self.bt, self.cl, self.maxL,
+                        self.w.scale, out=self.out, workspace=self.ws, kv_chunk_size=self.chunk_arg)
+
+    def store(self):
+        import paged_kv_cache_331_b200 as pa
+        pa.store_kvcache(self.nk, self.nv, self.kc, self.vc, self.slots)
+
+    def decode(self):
+        import paged_kv_cache_331_b200 as pa
+        pa.decode(self.q, self.kc, self.vc, self.bt, self.cl, self.maxL, self.w.scale, out=self.out,
+                  workspace=self.ws, kv_chunk_size=self.chunk_arg)
+
+
+def timed_launches(fn, reps, dev, before=None):
+    """Per-call CUDA-event times (ms) of fn on the current stream; `before` runs untimed ahead of each call."""
+    import torch
+    ev = []
+    for _ in range(reps):
+        if before is not None:
+            before()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(); fn(); b.record()
+        ev.append((a, b))
+    torch.cuda.synchronize(dev)
+    return [x.elapsed_time(y) for x, y in ev]
+
+
+def decode_roofline(d, ms, peaks, kernel):
+    """HBM roofline of one fused store + decode launch: algorithmic bytes / CUDA-event time."""
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    _, alg = decode_algorithmic_bytes(d.w)
+    alg += decode_store_bytes(d.w)
+    achieved = alg / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "algorithmic_bytes": alg, "launch_ms": round(ms, 5),
+            "peak_kind": f"HBM copy ({peaks.get('source')})"}
+
+
+def bench_decode_leg(name, desc, dev, peaks, reps, warmup):
+    """One decode workload on its own: store + decode launches timed one by one (inputs larger than L2 except
+    for the tiny workload, which is a latency case)."""
+    import paged_kv_cache_331_b200 as pa
+    from paged_kv_cache_331_b200 import workloads as W
+    import torch
+    w = W.WORKLOADS[name]()
+    d = DecodeOnDevice(w, dev)
+    for _ in range(warmup):
+        d.step()
+    if name == "tiny_decode":
+        # a latency case: 50 steps captured in one CUDA graph and replayed, so the device time per step is
+        # measured without the host's launch overhead (which dwarfs a kernel this small)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        n_graph = 50
+        with torch.cuda.graph(g):
+            for _ in range(n_graph):
+                d.step()
+        g.replay()
+        ms_all = [t / n_graph for t in timed_launches(g.replay, max(3, reps // n_graph), dev)]
+        eager = timed_launches(d.step, 20, dev)
+    else:
+        L2Flush(dev)()                 # the GPU stays busy while the host enqueues the first launches
+        ms_all = timed_launches(d.step, reps, dev)
+    assert pa.device_error() == 0
+    ms = float(np.mean(ms_all))
+    kv, _ = decode_algorithmic_bytes(w)
+    res = {"config": decode_config(w, desc), "reps": reps, "ms": round(ms, 5), "ms_median": round(float(np.median(ms_all)), 5),
+           "kv_gbs": round(kv / (ms / 1e3) / 1e9, 1), "seqs_per_s": round(w.num_seqs / (ms / 1e3), 1),
+           "kv_chunk_size": d.chunk, "launches_per_step": d.launches_per_step,
+           "roofline": decode_roofline(d, ms, peaks, "pa_store_decode")}
+    if name == "tiny_decode":
+        res["latency_us"] = round(ms * 1e3, 2)
+        res["eager_call_us"] = round(float(np.median(eager)) * 1e3, 2)
+        res["note"] = ("latency case (294 KB of KV, L2-resident): latency_us is the device time per step of 50 "
+                       "steps replayed from one CUDA graph; eager_call_us is one call from Python, host launch "
+                       "overhead included; parity is its bar")
+    return res, d
+
+
+def bench_store_rows(d, dev, reps, flush):
+    """store_kvcache of the workload's new rows on its own, L2 flushed (written, then evicted by a read) before
+    every rep: microseconds and GB/s (2 MB cannot fill HBM within a launch's lifetime)."""
+    import paged_kv_cache_331_b200 as pa
+    for _ in range(3):
+        d.store()
+    ms_all = timed_launches(d.store, reps, dev, before=flush)
+    assert pa.device_error() == 0
+    ms = float(np.median(ms_all))
+    nbytes = decode_store_bytes(d.w)
+    return {"rows": int(d.w.num_seqs), "us": round(ms * 1e3, 2), "bytes": nbytes,
+            "gbs": round(nbytes / (ms / 1e3) / 1e9, 1), "l2": "flushed before every rep"}
+
+
 def bench_decode(args, world, rank, dev, peaks):
+    """The headline: decode steps of the large-batch layer (256 sequences), timed as K consecutive steps."""
     import torch
     import paged_kv_cache_331_b200 as pa
     from paged_kv_cache_331_b200 import workloads as W
 
-    w = W.qwen3_decode(seed=2 + 1000 * rank)
-    q, kc, vc = to_dev(w.q, "bf16", dev), to_dev(w.k_cache, "bf16", dev), to_dev(w.v_cache, "bf16", dev)
-    nk, nv = to_dev(w.new_k, "bf16", dev), to_dev(w.new_v, "bf16", dev)
-    slots, bt, cl = to_dev(w.slot_mapping, "i32", dev), to_dev(w.block_tables, "i32", dev), to_dev(w.context_lens, "i32", dev)
-    out = torch.empty_like(q)
-    maxL = w.max_context_len
-    ws_bytes = pa.decode_workspace_size(w.num_seqs, w.num_heads, w.num_kv_heads, w.head_dim, maxL, w.block_size, 0)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    chunk = pa.decode_chunk_size(w.num_seqs, w.num_kv_heads, maxL, w.block_size)
-    # one launch per step: the new rows are stored by the decode kernel, whose last chunk CTA per
-    # (sequence, kv head) also merges the split-KV partials
-    launches_per_step = 1
-
-    def step():
-        pa.store_decode(q, nk, nv, slots, kc, vc, bt, cl, maxL, w.scale, out=out, workspace=ws)
-
+    w = W.large_batch_decode(seed=3 + 1000 * rank)
+    d = DecodeOnDevice(w, dev)
     for _ in range(args.warmup):
-        step()
+        d.step()
     torch.cuda.synchronize(dev)
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(dev.index, period_s=0.0002)
+    flush = L2Flush(dev)
     barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(dev.index) as clk:
+    with clk:
+        # the flush keeps the GPU busy while the host enqueues the first steps, so the timed region holds no
+        # launch gap; it is not part of the region
+        flush()
+        i0 = clk.mark()
         t0.record()
         for i in range(K):
             ev[i][0].record()
-            step()
+            d.step()
             ev[i][1].record()
         t1.record()
+        torch.cuda.synchronize(dev)
+        i1 = clk.mark()
+        # the same step as two calls (store kernel, then split + merge), for reference; the clock record goes on
+        # over these reps, which run the same HBM-bound kernels at the same clocks
+        Ku = max(3, min(K, 200))
+        evu = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Ku)]
+        for i in range(Ku):
+            evu[i][0].record()
+            d.store()
+            evu[i][1].record()
+            d.decode()
+            evu[i][2].record()
+        torch.cuda.synchronize(dev)
+        more = max(0, 40 - K)                       # keep the record going for at least ~8 ms of steps
+        for _ in range(more):
+            d.step()
         torch.cuda.synchronize(dev)
     barrier(world)
     elapsed_ms = t0.elapsed_time(t1)
     decode_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
     assert pa.device_error() == 0
     elapsed_ms = max_over_ranks(elapsed_ms, world)
-
-    # the same step as two calls (store kernel, then split + merge), for reference
-    Ku = max(3, min(K, 200))
-    evu = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Ku)]
-    for i in range(Ku):
-        evu[i][0].record()
-        pa.store_kvcache(nk, nv, kc, vc, slots)
-        evu[i][1].record()
-        pa.decode(q, kc, vc, bt, cl, maxL, w.scale, out=out, workspace=ws)
-        evu[i][2].record()
-    torch.cuda.synchronize(dev)
     unfused = {"store_ms": round(float(np.mean([e[0].elapsed_time(e[1]) for e in evu])), 5),
                "decode_ms": round(float(np.mean([e[1].elapsed_time(e[2]) for e in evu])), 5), "steps": Ku}
 
-    kv_bytes, alg_bytes = decode_algorithmic_bytes(w)
-    alg_bytes += decode_store_bytes(w)
+    kv_bytes, _ = decode_algorithmic_bytes(w)
     total_kv = sum_over_ranks(float(kv_bytes), world) * K
     value = total_kv / (elapsed_ms / 1e3) / 1e9
     seqs = sum_over_ranks(float(w.num_seqs), world) * K / (elapsed_ms / 1e3)
-    achieved = alg_bytes / (decode_ms / 1e3) / 1e9
-    traffic = profiled_traffic("decode")
+    roof = decode_roofline(d, decode_ms, peaks, "pa_store_decode (decode_split_kernel: store + decode)")
+    roof["traffic"] = profiled_traffic("decode")
 
     # end to end through host buffers: every step copies q, the new K/V rows and the metadata (one packed pinned
-    # buffer) to the device, runs the fused store + decode, and copies out back -- one CUDA graph
-    from paged_kv_cache_331_b200.graphs import HostDecodeStep
-    hstep = HostDecodeStep(kc, vc, w.num_seqs, w.num_heads, w.block_tables.shape[1], maxL, w.scale)
-    hin = hstep.inputs()
-    for name, arr in (("q", w.q), ("new_k", w.new_k), ("new_v", w.new_v)):
-        hin[name].view(torch.int16).copy_(torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)))
-    hin["slot_mapping"].copy_(torch.from_numpy(w.slot_mapping))
-    hin["block_tables"].copy_(torch.from_numpy(w.block_tables))
-    hin["context_lens"].copy_(torch.from_numpy(w.context_lens))
-    h2d, d2h = hstep.h2d_bytes, hstep.d2h_bytes
+    # buffer) to the device, runs the fused store + decode, and copies out back; the host waits for each step's
+    # output one step behind, so a step's copies overlap the neighbouring steps' kernels
+    from paged_kv_cache_331_b200.graphs import HostDecodePipeline
+    pipe = HostDecodePipeline(d.kc, d.vc, w.num_seqs, w.num_heads, w.block_tables.shape[1], d.maxL, w.scale,
+                              depth=3)
+    for s in range(pipe.depth):
+        hin = pipe.inputs(s)
+        for name, arr in (("q", w.q), ("new_k", w.new_k), ("new_v", w.new_v)):
+            hin[name].view(torch.int16).copy_(torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)))
+        hin["slot_mapping"].copy_(torch.from_numpy(w.slot_mapping))
+        hin["block_tables"].copy_(torch.from_numpy(w.block_tables))
+        hin["context_lens"].copy_(torch.from_numpy(w.context_lens))
 
-    def e2e_step():
-        hstep.run()
+    def e2e_run(n):
+        tickets = []
+        for i in range(n):
+            if i >= pipe.depth:
+                pipe.wait(tickets[i - pipe.depth])
+            tickets.append(pipe.submit())
+        for t in tickets[max(0, n - pipe.depth):]:
+            pipe.wait(t)
 
-    for _ in range(min(args.warmup, 10)):
-        e2e_step()
+    e2e_run(max(3, min(args.warmup, 10)))
     Ke = max(1, min(K, 500))
     barrier(world)
     torch.cuda.synchronize(dev)
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush()
     s0.record()
-    for _ in range(Ke):
-        e2e_step()
+    e2e_run(Ke)
+    pipe.join()
     s1.record()
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
     e2e_value = sum_over_ranks(float(kv_bytes), world) * Ke / (e2e_ms / 1e3) / 1e9
+    assert pa.device_error() == 0
+    clocks = clk.summary()
+    clocks["window"] = ("the K timed steps, then the unfused reps and further steps of the same workload "
+                        "(the same HBM-bound kernel)")
+    clocks["timed_region"] = clk.summary(i0, i1)
 
-    return w, {
+    return w, d, {
         "value": value, "ms_per_step": elapsed_ms / K, "seqs_per_s": seqs, "unfused": unfused,
-        "decode_ms": decode_ms, "kv_bytes_per_step": kv_bytes, "alg_bytes": alg_bytes, "achieved": achieved,
-        "traffic": traffic, "chunk": chunk, "ws_bytes": ws_bytes, "launches": launches_per_step * K,
-        "clocks": clk.summary(), "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                                         "d2h_bytes_per_step": d2h, "steps": Ke},
+        "decode_ms": decode_ms, "kv_bytes_per_step": kv_bytes, "roofline": roof,
+        "chunk": d.chunk, "ws_bytes": d.ws_bytes, "launches": d.launches_per_step * K,
+        "clocks": clocks, "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": pipe.h2d_bytes,
+                                  "d2h_bytes_per_step": pipe.d2h_bytes, "steps": Ke,
+                                  "how": "pinned host buffers; per step one H2D copy of the packed inputs, the fused "
+                                         "store + decode, one D2H copy of out; three buffer slots on three streams so a "
+                                         "step's copies overlap the neighbouring steps' kernels; the host waits for "
+                                         "every step's output"},
     }
 
 
@@ -584,42 +751,52 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local if world > 1 else 0)
     import paged_kv_cache_331_b200 as pa
     pa.lib()
-    w, d = bench_decode(args, world, rank, dev, peaks)
+    w, d, res = bench_decode(args, world, rank, dev, peaks)
+    legs, store3 = None, None
+    if rank == 0 and not args.no_legs:
+        flush = L2Flush(dev)
+        store3 = bench_store_rows(d, dev, max(10, min(args.steps, 100)), flush)
+        del d, flush
+        torch.cuda.empty_cache()
+        legs = {}
+        for name, desc in DECODE_LEGS.items():
+            reps = max(50, min(args.steps, 500)) if name != "tiny_decode" else 200
+            legs[name], dl = bench_decode_leg(name, desc, dev, peaks, reps, max(3, args.warmup))
+            del dl
+            torch.cuda.empty_cache()
     pre = bench_prefill(args, dev, peaks) if (rank == 0 and not args.no_prefill) else None
     gr = bench_graph(args, dev) if (rank == 0 and not args.no_graph) else None
     cpu = cpu_baseline(w) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if rank != 0:
         return
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    config = decode_config(w, HEADLINE[1])
+    config["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
     line = {
-        "metric": METRIC, "value": round(d["value"], 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(d["ms_per_step"], 5), "higher_is_better": True,
+        "metric": METRIC, "value": round(res["value"], 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(res["ms_per_step"], 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32",
         "data": "synthetic: seeded N(0,1) bf16 Q/K/V, block tables drawn from a shuffled 1.25x pool",
-        "config": {"workload": w.name, "num_seqs": w.num_seqs, "context_lens": "U[128,4096]",
-                   "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
-                   "block_size": w.block_size, "pool_blocks": w.num_blocks, "kv_bytes_per_step": d["kv_bytes_per_step"],
-                   "step": "store of the 64 new rows + decode (split-KV, merged in-kernel): one pa_store_decode launch",
-                   "kv_chunk_size": d["chunk"],
-                   "l2": f"inputs larger than L2: {d['kv_bytes_per_step'] / 1e6:.0f} MB KV per step vs 126 MB L2",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "seqs_per_s": round(d["seqs_per_s"], 1),
-        "hbm_frac": round(d["value"] / world / hbm, 4),
-        "roofline": {"bound": "hbm", "kernel": "pa_store_decode (decode_split_kernel: store + split + merge)",
-                     "achieved": round(d["achieved"], 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(d["achieved"] / hbm, 4), "traffic": d["traffic"],
-                     "algorithmic_bytes": d["alg_bytes"], "launch_ms": round(d["decode_ms"], 5),
-                     "peak_kind": f"HBM copy ({peaks.get('source')})"},
-        "unfused_step": d["unfused"],
-        "e2e": d["e2e"], "gpu_launches": d["launches"], "clocks": d["clocks"],
+        "config": config,
+        "step": f"store of the {w.num_seqs} new rows + decode of every sequence: one pa_store_decode launch "
+                f"(kv_chunk_size {res['chunk']})",
+        "seqs_per_s": round(res["seqs_per_s"], 1),
+        "hbm_frac": round(res["value"] / world / hbm, 4),
+        "roofline": res["roofline"],
+        "unfused_step": res["unfused"],
+        "e2e": res["e2e"], "gpu_launches": res["launches"], "clocks": res["clocks"],
     }
+    if store3 is not None:
+        line["store_256_rows"] = store3
+    if legs is not None:
+        line["decode_workloads"] = legs
     if pre is not None:
         line["prefill"] = pre
     if gr is not None:
         line["graph"] = gr
     if cpu is not None:
         line["cpu_baseline"] = cpu
-        line["speedup_vs_cpu_baseline"] = round(d["value"] / cpu["value"], 1)
+        line["speedup_vs_cpu_baseline"] = round(res["value"] / cpu["value"], 1)
     print(json.dumps(line), flush=True)
 
 
@@ -632,13 +809,14 @@ def run_reference(args, world, rank):
     from oracle import oracle as O
     from paged_kv_cache_331_b200 import workloads as W
     orc = O.get()
-    w = W.qwen3_decode()
+    w = W.large_batch_decode()
     # calibrate: sequences per step so that warmup + steps end within about --reference-seconds
     one = W.decode_workload(w.context_lens[:1], w.num_heads, w.num_kv_heads, w.head_dim, w.block_size,
                             rng=np.random.default_rng(0))
     t = time.perf_counter()
     orc.decode(one.q, one.k_cache, one.v_cache, one.block_tables, one.context_lens, one.scale)
-    t1 = max(time.perf_counter() - t, 1e-4) * max(1.0, 2112.0 / float(one.context_lens[0]))
+    mean_len = float(w.context_lens.mean())
+    t1 = max(time.perf_counter() - t, 1e-4) * max(1.0, mean_len / float(one.context_lens[0]))
     per_step_budget = args.reference_seconds / max(1, args.steps + args.warmup)
     nseq = int(max(1, min(w.num_seqs, per_step_budget / t1)))
     sub = slice(0, nseq)
@@ -657,14 +835,14 @@ def run_reference(args, world, rank):
     kv = int(w.context_lens[sub].astype(np.int64).sum()) * w.num_kv_heads * w.head_dim * 4
     value = kv * args.steps / el / 1e9
     sample = f"first {nseq} of {w.num_seqs} sequences per step (store + decode)"
+    config = decode_config(w, HEADLINE[1])
+    config["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic: seeded N(0,1) bf16 Q/K/V, block tables drawn from a shuffled 1.25x pool",
-        "config": {"workload": w.name, "num_seqs": w.num_seqs, "context_lens": "U[128,4096]",
-                   "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
-                   "block_size": w.block_size, "sample": sample},
+        "config": config,
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": orc.max_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -681,6 +859,8 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="skip the per-workload decode legs (tiny, Qwen3-shaped, long context) and the row store")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
                     help="--impl reference: about how long the oracle's warm-up and timed steps take together")
     ap.add_argument("--no-prefill-clock", action="store_true",

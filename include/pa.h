@@ -36,9 +36,13 @@
  *   PA_ERR_UNSUPPORTED for legal shapes this build has no kernel for,
  *   PA_ERR_WORKSPACE for a workspace that is too small, PA_ERR_CUDA when a
  *   launch fails (pa_last_error() then holds the CUDA message).
- * - Device-side contract (not checked on the device): block ids in the used
- *   part of block_tables lie in [0, num_blocks); slots are unique;
- *   context_lens[b] <= max_context_len and <= max_blocks_per_seq*block_size.
+ * - Device-side contract: block ids in the used part of block_tables lie in
+ *   [0, num_blocks); slots are unique; context_lens[b] <= max_context_len and
+ *   <= max_blocks_per_seq*block_size; cu_seqlens_q/k agree with total_q,
+ *   max_seqlen_q/k and the table width.  The kernels check every one of
+ *   these that could send an access outside the caller's buffers, skip or
+ *   clamp that access and record a code (pa_device_error); uniqueness of
+ *   slots is not checked.
  * - Supported: head_dim 64 or 128; num_heads a multiple of num_kv_heads
  *   with group size G = num_heads / num_kv_heads in 1..8 for decode and
  *   G in {1, 2, 4, 8} for prefill; block_size a power of two in [16, 1024];
@@ -88,8 +92,8 @@ PA_API int32_t pa_version(void);
  *   k_cache[s / block_size][s % block_size][:][:] = key[t][:][:]
  *   v_cache[s / block_size][s % block_size][:][:] = value[t][:][:]
  * A bit copy.  Slots equal to -1 are skipped; a slot outside
- * [0, num_blocks*block_size) other than -1 breaks the contract and is also
- * skipped, never written out of bounds.
+ * [0, num_blocks*block_size) other than -1 breaks the contract: it is also
+ * skipped, never written out of bounds, and device error code 6 is recorded.
  *
  * key, value:    [num_tokens, num_kv_heads, head_dim] bf16, row t starting at
  *                element t*key_row_stride (t*value_row_stride); the strides
@@ -140,7 +144,8 @@ PA_API pa_status pa_rotary_cos_sin_cache(float* table, int32_t max_position, int
  * key, value:    as for pa_store_kvcache.
  * positions:     [num_tokens] int32 in [0, max_position).  A position
  *                outside that range leaves the token's q_out rows and K cache
- *                rows unwritten and sets device error code 4.
+ *                rows unwritten and sets device error code 4.  A slot outside
+ *                the cache (other than -1) is skipped and sets code 6.
  * cos_sin_cache: [max_position, head_dim] float as pa_rotary_cos_sin_cache
  *                fills it.
  * Requires head_dim 64 or 128, every pointer 16-byte aligned and every row
@@ -199,7 +204,9 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int3
  * q, out:         [num_seqs, num_heads, head_dim] bf16 (dense).
  * block_tables:   [num_seqs, max_blocks_per_seq] int32; entries past
  *                 ceil(L/block_size) are never read (may be -1).
- * context_lens:   [num_seqs] int32, each <= max_context_len.
+ * context_lens:   [num_seqs] int32, each <= max_context_len and <=
+ *                 max_blocks_per_seq*block_size; a larger (or negative) one
+ *                 is clamped into that range and sets device error code 7.
  * kv_chunk_size:  0 = automatic; otherwise tokens per split-KV chunk, a
  *                 multiple of 64 (a value >= max_context_len disables the
  *                 split).  Sequences longer than one chunk are processed by
@@ -239,7 +246,10 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
  *   the last call's contents; nothing needs it zeroed, since every partial a
  *   call reads is written earlier in that call.
  * - The array's device address is looked up on the first call made on each
- *   device; make that first call before any stream capture starts.
+ *   device; make that first call before any stream capture starts.  A
+ *   successful lookup is kept until the library is unloaded (it is stale
+ *   after a reset of the device's primary context, e.g. cudaDeviceReset); a
+ *   failed one is retried on the next call.
  */
 #define PA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 
@@ -265,10 +275,9 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache
  * error code 5.  key/value rows must be 16-byte aligned with strides that are
  * multiples of 8 elements (PA_ERR_UNSUPPORTED otherwise).  Every other
  * argument, the workspace rule and the errors are pa_decode's.
- * Precondition the kernel does not check: the block-table entry that covers
- * position context_lens[b]-1 is a valid block id (< num_blocks); the row is
- * written at the slot that entry names.  (pa_store_kvcache skips a slot
- * outside the cache instead.)
+ * The row is written at the slot the block-table entry for position
+ * context_lens[b]-1 names; if that entry lies outside the cache the row is
+ * not written and device error code 6 is recorded.
  */
 PA_API pa_status pa_store_decode(void* out, const void* q, const void* key, const void* value, int64_t key_row_stride,
                           int64_t value_row_stride, const int32_t* slot_mapping, void* k_cache, void* v_cache,
@@ -335,11 +344,12 @@ PA_API pa_status pa_merge_partials(void* out, const float* o_parts, const float*
  * max_seqlen_q/k: upper bounds of Lq and Lk over the batch.
  * block_tables:   as for pa_decode, entries past ceil(Lk/block_size) unread.
  *
- * Preconditions on device data that the kernel does not check: total_q and
- * max_seqlen_q/k agree with cu_seqlens_q/k, and Lk <= max_blocks_per_seq *
- * block_size.  A violation can read or write outside the caller's buffers.
- * (pa_decode, by contrast, clamps each context length to max_context_len and
- * to the table width.)
+ * Checked on the device: a sequence whose cu_seqlens_q/k disagree with
+ * total_q, max_seqlen_q/k or the table width (Lk > max_blocks_per_seq *
+ * block_size) is skipped, its output rows left unwritten, and device error
+ * code 8 is recorded; a used block-table entry outside the cache records
+ * code 6 and reads zeros.  Nothing is read or written outside the caller's
+ * buffers.
  */
 PA_API pa_status pa_prefill_varlen(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int32_t total_q,
@@ -355,10 +365,26 @@ PA_API pa_status pa_prefill_varlen(void* out, const void* q, const void* k_cache
  * and pa_rotary_store_kvcache sets it for a position outside its table.
  * Codes: 0 none, 1 a pipeline wait timed out, 2 the wait for in-flight copies
  * at exit timed out, 3 dynamic shared memory misaligned, 4 rotary position
- * out of range, 5 a pa_store_decode slot that is not the new token's.
- * Diagnostic only.
+ * out of range, 5 a pa_store_decode slot that is not the new token's,
+ * 6 a slot (other than -1) or a used block-table entry outside the cache
+ * (the store is skipped; decode and prefill read zeros for that block),
+ * 7 a decode context length above max_context_len or the table width (it is
+ * clamped), 8 a prefill sequence whose cu_seqlens_q/k disagree with
+ * total_q, max_seqlen_q/k or the table width (that sequence is skipped: its
+ * output rows are not written).  The first code recorded since the last
+ * read wins.  Diagnostic only.
  */
 PA_API pa_status pa_device_error(int32_t* code_out, void* stream);
+
+/*
+ * pa_selftest_wait_timeout -- launch one CTA whose pipeline wait has nothing
+ * to arrive on, to check the time-limited waits the kernels rely on.  The
+ * wait gives up after limit_ns nanoseconds (1e3 .. 1e9) and records code 1
+ * in the device error word (pa_device_error); the CTA then frees the tensor
+ * memory it allocated and returns, as the kernels do on that path.  Nothing
+ * hangs and nothing faults; later launches are unaffected.  Diagnostic only.
+ */
+PA_API pa_status pa_selftest_wait_timeout(int64_t limit_ns, void* stream);
 
 #ifdef __cplusplus
 }

@@ -15,9 +15,9 @@ touch CUDA.  ``workloads`` builds seeded synthetic inputs.
 """
 from ._binding import (PagedAttentionError, decode, decode_chunk_size, decode_chunk_size_for, decode_noalloc,
                        decode_partial, decode_workspace_size, device_error, lib, merge_partials, prefill_varlen, rotary_cos_sin_cache,
-                       rotary_store_kvcache, store_decode, store_kvcache)
+                       rotary_store_kvcache, selftest_wait_timeout, store_decode, store_kvcache)
 
 __all__ = ["store_kvcache", "rotary_cos_sin_cache", "rotary_store_kvcache", "decode", "decode_noalloc",
            "decode_partial", "merge_partials", "store_decode",
-           "prefill_varlen", "decode_workspace_size", "decode_chunk_size", "decode_chunk_size_for", "device_error", "PagedAttentionError",
+           "prefill_varlen", "decode_workspace_size", "decode_chunk_size", "decode_chunk_size_for", "device_error", "selftest_wait_timeout", "PagedAttentionError",
            "lib"]

@@ -42,6 +42,7 @@ _PROTOS = {
                                                _i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "pa_decode_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                          _f32, _i32, _vp]),
+    "pa_selftest_wait_timeout": (ctypes.c_int, [_i64, _vp]),
 }
 
 
@@ -237,7 +238,8 @@ def store_decode(q, key, value, slot_mapping, k_cache, v_cache, block_tables, co
     """pa_store_decode: store each sequence's new K/V row (slot of position L-1, or -1) and decode, one launch.
 
     ``validate=True`` first checks on the host (a synchronising copy) that every slot is the one its block table
-    names for the newest position, through a valid block id: the kernel takes that on trust."""
+    names for the newest position, through a valid block id, and raises before the launch.  Without it the kernel
+    still skips a slot that breaks this and records device error code 5 or 6 (read with ``device_error()``)."""
     for n, t in (("q", q), ("key", key), ("value", value), ("k_cache", k_cache), ("v_cache", v_cache)):
         _cuda(t, n, torch.bfloat16)
     for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
@@ -369,8 +371,10 @@ def prefill_varlen(q, k_cache, v_cache, cu_seqlens_q, cu_seqlens_k, max_seqlen_q
                    causal=True, *, out=None, stream=None, validate=False):
     """Varlen prefill over the paged cache: q [total_q, Hq, D] -> out [total_q, Hq, D].
 
-    ``validate=True`` first checks on the host (a synchronising copy) what the kernel takes on trust: the
-    cu_seqlens agree with total_q, max_seqlen_q/k and the block tables, whose entries are valid block ids."""
+    ``validate=True`` first checks on the host (a synchronising copy) that the cu_seqlens agree with total_q,
+    max_seqlen_q/k and the block tables, whose entries are valid block ids, and raises before the launch.  Without
+    it the kernel still skips a sequence whose metadata breaks this (device error code 8) and reads zeros for a
+    block id outside the cache (code 6)."""
     for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _cuda(t, n, torch.bfloat16); _dense(t, n)
     for n, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k), ("block_tables", block_tables)):
@@ -410,3 +414,12 @@ def device_error(stream=None, device=None) -> int:
         s = stream.cuda_stream if stream is not None else torch.cuda.current_stream(dev).cuda_stream
         _check(lib().pa_device_error(ctypes.byref(code), s), "pa_device_error")
     return int(code.value)
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None, device=None) -> None:
+    """Launch the one-CTA kernel whose pipeline wait has nothing to arrive on: it gives up after limit_ns,
+    records code 1 (read it with device_error()), frees its tensor memory and returns."""
+    dev = device if device is not None else torch.cuda.current_device()
+    with torch.cuda.device(dev):
+        s = stream.cuda_stream if stream is not None else torch.cuda.current_stream(dev).cuda_stream
+        _check(lib().pa_selftest_wait_timeout(int(limit_ns), s), "pa_selftest_wait_timeout")

@@ -81,6 +81,8 @@ struct DecodeParams {
   const int32_t* slot_mapping;
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
+  int64_t num_slots;        // num_blocks * block_size: a slot at or past it is outside the cache
+  int32_t num_blocks;
 };
 
 // Per-shape configuration.  Two CTAs share an SM whenever their shared memory
@@ -185,7 +187,9 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
 
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int L = clamp_context(__ldg(p.context_lens + b), p);
+  const int L_raw = __ldg(p.context_lens + b);
+  const int L = clamp_context(L_raw, p);
+  if (L != L_raw && chunk == 0 && g == 0 && threadIdx.x == 0) record_error(p.err, kErrContextLen);
   const int hq0 = g * G;
 
   if (L == 0) {   // no keys: the output is defined as zero (a partial: 0 with lse = -inf)
@@ -219,13 +223,15 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
     if (p.slot_mapping && chunk == nchunks - 1) {
       // Fused store: this CTA is the only reader of position L-1 (its last
       // tile), so it writes the new token's K/V row of kv head g into the
-      // cache before loading any tile.  The slot must be that position's;
-      // any other slot (but -1) is reported and not written.
+      // cache before loading any tile.  The slot must be that position's
+      // (any other slot but -1 is reported and not written) and lie inside
+      // the cache (a table entry past the cache is reported, not followed).
       const int32_t slot = __ldg(p.slot_mapping + b);
       const int32_t* btb = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq;
       const int pos = L - 1;
       const int64_t expect = static_cast<int64_t>(__ldg(btb + pos / p.block_size)) * p.block_size + pos % p.block_size;
-      if (slot >= 0 && slot == expect) {
+      const bool inside = slot >= 0 && slot < p.num_slots;
+      if (slot == expect && inside) {
         constexpr int kLanesPerRow = D / 8;   // 16-byte pieces of one head row
         if (lane < 2 * kLanesPerRow) {
           const bool is_v = lane >= kLanesPerRow;
@@ -238,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
           fence_proxy_async_global();
         }
       } else if (slot != -1 && lane == 0) {
-        record_error(p.err, kErrBadSlot);
+        record_error(p.err, slot == expect ? kErrOutOfCache : kErrBadSlot);
       }
       __syncwarp();
     }
@@ -259,6 +265,10 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
         for (int k = 0; k < nbox; ++k) {
           const int tok = t0 + k * p.box_rows;
           const int blk = __ldg(bt + (tok >> bs_shift));
+          // a table entry outside the cache is reported; TMA fills the box's
+          // rows outside the tensor map with zeros, so nothing outside the
+          // cache is read
+          if (static_cast<unsigned>(blk) >= static_cast<unsigned>(p.num_blocks)) record_error(p.err, kErrOutOfCache);
           const int row = (blk << bs_shift) + (tok & (p.block_size - 1));
           const size_t soff = (static_cast<size_t>(s) * kTile + static_cast<size_t>(k) * p.box_rows) * D;
           tma_load_3d_hint(sK + soff, &tmK, &full[s], 0, g, row, pol);
@@ -687,6 +697,8 @@ pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.slot_mapping = a.slot_mapping;
   p.k_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(a.k_cache));
   p.v_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(a.v_cache));
+  p.num_slots = static_cast<int64_t>(a.num_blocks) * a.block_size;
+  p.num_blocks = a.num_blocks;
   static std::atomic<uint32_t> launches{0};
   const bool fused_merge = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads <= kMergeCounters;
   p.merge_slot = (a.max_chunks > 1 && fused_merge) ? static_cast<int32_t>(launches.fetch_add(1) % kMergeSlots) : -1;

@@ -18,7 +18,10 @@
 //    earlier in the same call.
 //  * The device address of the array is looked up on the first call made on
 //    each device (with that device current); that first call should happen
-//    before any stream capture begins on the device.
+//    before any stream capture begins on the device.  The address is kept
+//    until the library is unloaded, so it is stale after the device's
+//    primary context is reset (cudaDeviceReset); a lookup that failed is
+//    tried again on the next call.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -36,11 +39,12 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_status[kMaxDevices];
-std::once_flag g_scratch_once[kMaxDevices];
+std::mutex g_scratch_mutex;
 
-// Device address of the scratch array on the current device (looked up once
-// per device).  Returns nullptr and records a message on failure.
+// Device address of the scratch array on the current device.  A successful
+// lookup is kept for the library's lifetime (it stays valid until the
+// device's primary context is reset); a failed one is not kept, so the next
+// call tries again.  Returns nullptr and records a message on failure.
 void* scratch_for_current_device() {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -52,15 +56,15 @@ void* scratch_for_current_device() {
     set_last_error("decode_noalloc: device ordinal %d is beyond the %d this build tracks", dev, kMaxDevices);
     return nullptr;
   }
-  std::call_once(g_scratch_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
     void* ptr = nullptr;
-    g_scratch_status[dev] = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-    g_scratch_ptr[dev] = g_scratch_status[dev] == cudaSuccess ? ptr : nullptr;
-  });
-  if (g_scratch_status[dev] != cudaSuccess || !g_scratch_ptr[dev]) {
-    set_last_error("decode_noalloc: cudaGetSymbolAddress failed on device %d: %s", dev,
-                   cudaGetErrorString(g_scratch_status[dev]));
-    return nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess || !ptr) {
+      set_last_error("decode_noalloc: cudaGetSymbolAddress failed on device %d: %s", dev, cudaGetErrorString(e));
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = ptr;
   }
   return g_scratch_ptr[dev];
 }

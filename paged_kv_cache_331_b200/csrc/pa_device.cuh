@@ -18,6 +18,9 @@ enum DeviceErrorCode : unsigned int {
   kErrSmemAlign = 3,       // dynamic shared memory not 1024-byte aligned
   kErrBadPosition = 4,     // a rotary position outside [0, max_position)
   kErrBadSlot = 5,         // fused store + decode: a slot that is not the new token's position
+  kErrOutOfCache = 6,      // a slot or block-table entry outside the cache: that access is skipped
+  kErrContextLen = 7,      // a decode context length above max_context_len or the table width (clamped)
+  kErrPrefillMeta = 8,     // prefill metadata at odds with total_q, max_seqlen_q/k or the table width
 };
 
 #ifndef PA_WAIT_LIMIT_NS
@@ -72,16 +75,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (and records `code`) if that takes longer than PA_WAIT_LIMIT_NS.
+// (and records `code`) if that takes longer than limit_ns (PA_WAIT_LIMIT_NS
+// unless a caller asks for less).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* err,
-                                          unsigned int code = kErrWaitTimeout) {
+                                          unsigned int code = kErrWaitTimeout,
+                                          uint64_t limit_ns = PA_WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > PA_WAIT_LIMIT_NS) {
+    if (global_timer_ns() - t0 > limit_ns) {
       record_error(err, code);
       return false;
     }
@@ -91,8 +96,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
 // Warp-uniform variant: every lane of the warp calls it and all agree on the
 // outcome, so code after it (tcgen05 .sync.aligned instructions) never runs
 // diverged.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, unsigned int* err) {
-  const bool ok = mbar_wait(bar, parity, err);
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, unsigned int* err,
+                                               uint64_t limit_ns = PA_WAIT_LIMIT_NS) {
+  const bool ok = mbar_wait(bar, parity, err, kErrWaitTimeout, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -91,6 +91,10 @@ struct PrefillParams {
   unsigned int* err;
   int32_t sched_slot;
   int32_t out_v8;            // out is 32-byte aligned: write 32-byte vectors
+  int32_t total_q;           // rows of q / out
+  int32_t max_seqlen_q;
+  int32_t max_seqlen_k;
+  int32_t num_blocks;
 };
 
 template <int D>
@@ -180,6 +184,7 @@ struct Item {
   int b, g;
   int Lq, Lk, q_row0, pos_off;
   bool valid, has_b;
+  bool bad;                               // the sequence's metadata breaks the call's contract: skipped
   int qtA, qtB, ntA, ntB, fullA, fullB;   // query tile, key tiles, keys every row sees
 };
 
@@ -190,16 +195,25 @@ __device__ __forceinline__ Item decode_item(int t, int num_seqs, int num_kv_head
   const int rank = t / per_rank;
   it.b = (t % per_rank) / num_kv_heads;
   it.g = t % num_kv_heads;
-  const int cq0 = __ldg(p.cu_seqlens_q);
-  const int cqb = __ldg(p.cu_seqlens_q + it.b);
-  it.Lq = __ldg(p.cu_seqlens_q + it.b + 1) - cqb;
-  it.Lk = __ldg(p.cu_seqlens_k + it.b + 1) - __ldg(p.cu_seqlens_k + it.b);
-  it.q_row0 = cqb - cq0;
+  const int64_t cq0 = __ldg(p.cu_seqlens_q);
+  const int64_t cqb = __ldg(p.cu_seqlens_q + it.b);
+  const int64_t lq = __ldg(p.cu_seqlens_q + it.b + 1) - cqb;
+  const int64_t lk = __ldg(p.cu_seqlens_k + it.b + 1) - __ldg(p.cu_seqlens_k + it.b);
+  const int64_t row0 = cqb - cq0;
+  // Metadata that would make the item read or write outside the caller's
+  // buffers (rows past total_q, keys past the block-table row) or miss rows
+  // (more query tokens than max_seqlen_q provides items for) is reported and
+  // the sequence is skipped.
+  it.bad = lq < 0 || lk < lq || lq > p.max_seqlen_q || lk > p.max_seqlen_k ||
+           lk > static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size || row0 < 0 || row0 + lq > p.total_q;
+  it.Lq = it.bad ? 0 : static_cast<int>(lq);
+  it.Lk = it.bad ? 0 : static_cast<int>(lk);
+  it.q_row0 = it.bad ? 0 : static_cast<int>(row0);
   it.pos_off = it.Lk - it.Lq;
   const int ntq = (it.Lq + QP - 1) / QP;
   const int npairs = (ntq + 1) / 2;
   const int pair = npairs - 1 - rank;
-  it.valid = pair >= 0 && it.Lk >= it.Lq && it.Lk > 0;
+  it.valid = !it.bad && pair >= 0 && it.Lk >= it.Lq && it.Lk > 0;
   it.has_b = it.valid && 2 * pair + 1 < ntq;
   it.qtA = it.has_b ? 2 * pair + 1 : 2 * pair;
   it.qtB = 2 * pair;
@@ -319,6 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           t = static_cast<int>(atomicAdd(next_item, 1u));
           if (t >= num_items) break;
           it = decode_item<QP>(t, num_seqs, num_kv_heads, p);
+          if (it.bad) record_error(p.err, kErrPrefillMeta);
         } while (!it.valid);
         const int q = n % kWorkQ;
         if (!(ok = mbar_wait(&work_empty[q], ((n / kWorkQ) & 1) ^ 1, p.err))) break;
@@ -337,6 +352,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < nbox; ++k) {
             const int tok = j * kBN + k * p.box_rows;
             const int blk = __ldg(bt + (tok >> bs_shift));
+            // a table entry outside the cache is reported; TMA fills rows
+            // outside the tensor map with zeros, so nothing outside is read
+            if (static_cast<unsigned>(blk) >= static_cast<unsigned>(p.num_blocks)) record_error(p.err, kErrOutOfCache);
             const int row = (blk << bs_shift) + (tok & (p.block_size - 1));
             for (int c = 0; c < kChunks; ++c)
               tma_load_3d(dst + c * kChunkBytes + k * p.box_rows * 128, map, bar, c * 64, it.g, row);
@@ -713,6 +731,10 @@ pa_status launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.err = current_device_info()->error_word;
   p.out_v8 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
+  p.total_q = a.total_q;
+  p.max_seqlen_q = a.max_seqlen_q;
+  p.max_seqlen_k = a.max_seqlen_k;
+  p.num_blocks = a.num_blocks;
   static std::atomic<uint32_t> launches{0};
   p.sched_slot = static_cast<int32_t>(launches.fetch_add(1) % kSchedSlots);
   // persistent grid: at most one CTA per SM, each walking every gridDim.x-th work item

@@ -68,7 +68,10 @@ __global__ void __launch_bounds__(kRotThreads) rotary_store_kernel(RotaryArgs a,
 
   if (r >= a.num_heads + a.num_kv_heads) {   // value row: a copy into the slot
     const int32_t slot = __ldg(a.slot_mapping + t);
-    if (slot < 0 || slot >= a.num_slots) return;
+    if (slot < 0 || slot >= a.num_slots) {   // -1: skip; anything else is reported, never written
+      if (slot != -1 && j == 0) record_error(err, kErrOutOfCache);
+      return;
+    }
     const int h = r - a.num_heads - a.num_kv_heads;
     const uint16_t* src = static_cast<const uint16_t*>(a.value) + t * a.value_row_stride + static_cast<int64_t>(h) * D;
     uint16_t* dst = static_cast<uint16_t*>(a.v_cache) + slot * kv_row + static_cast<int64_t>(h) * D;
@@ -83,7 +86,10 @@ __global__ void __launch_bounds__(kRotThreads) rotary_store_kernel(RotaryArgs a,
   int32_t slot = 0;
   if (!is_q) {
     slot = __ldg(a.slot_mapping + t);
-    if (slot < 0 || slot >= a.num_slots) return;
+    if (slot < 0 || slot >= a.num_slots) {
+      if (slot != -1 && j == 0) record_error(err, kErrOutOfCache);
+      return;
+    }
   }
   const int32_t pos = __ldg(a.positions + t);
   if (pos < 0 || pos >= a.max_position) {

@@ -36,14 +36,17 @@ template <typename V>
 __global__ void __launch_bounds__(kStoreThreads) store_kvcache_kernel(
     const V* __restrict__ key, const V* __restrict__ value, int64_t key_stride_units, int64_t value_stride_units,
     V* __restrict__ k_cache, V* __restrict__ v_cache, const int32_t* __restrict__ slot_mapping, int32_t num_tokens,
-    int32_t row_units, int64_t num_slots) {
+    int32_t row_units, int64_t num_slots, unsigned int* __restrict__ err) {
   const int64_t wid = (static_cast<int64_t>(blockIdx.x) * kStoreThreads + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= 2 * static_cast<int64_t>(num_tokens)) return;
   const int64_t t = wid >> 1;
   const bool is_v = wid & 1;
   const int32_t slot = __ldg(slot_mapping + t);
-  if (slot < 0 || slot >= num_slots) return;   // -1: skip; anything else out of range: never written
+  if (slot < 0 || slot >= num_slots) {   // -1: skip; anything else out of range is reported, never written
+    if (slot != -1 && lane == 0) record_error(err, kErrOutOfCache);
+    return;
+  }
   const V* src = is_v ? value + t * value_stride_units : key + t * key_stride_units;
   V* dst = (is_v ? v_cache : k_cache) + static_cast<int64_t>(slot) * row_units;
   for (int base = 0; base < row_units; base += 32 * kMaxChunksPerLane) {
@@ -71,7 +74,7 @@ cudaError_t launch_typed(const void* key, const void* value, int64_t key_row_str
   store_kvcache_kernel<V><<<static_cast<unsigned>(blocks), kStoreThreads, 0, stream>>>(
       static_cast<const V*>(key), static_cast<const V*>(value), key_row_stride / kElemsPerUnit,
       value_row_stride / kElemsPerUnit, static_cast<V*>(k_cache), static_cast<V*>(v_cache), slot_mapping,
-      num_tokens, row_elems / kElemsPerUnit, num_slots);
+      num_tokens, row_elems / kElemsPerUnit, num_slots, current_device_info()->error_word);
   return cudaGetLastError();
 }
 

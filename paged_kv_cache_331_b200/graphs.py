@@ -200,3 +200,137 @@ class HostDecodeStep:
         self.graph.replay()
         torch.cuda.current_stream(self.out.device).synchronize()
         return self.host_out
+
+
+class HostDecodePipeline:
+    """Decode steps fed from and returned to host memory, with the copies of
+    one step overlapping the kernels of its neighbours.
+
+    A serving loop that gets each step's inputs from the host and hands each
+    output back pays, per step, a host-to-device copy, the kernel and a
+    device-to-host copy.  Run back to back on one stream they add up.  Here
+    each of the ``depth`` slots has its own pinned and device buffers, and
+    the three parts run on three streams:
+
+        h2d stream:  copy inputs of step i (slot i % depth)
+        compute:     pa_store_decode of step i (a CUDA graph per slot), after
+                     that copy and after the output copy of step i - depth
+        d2h stream:  copy the output of step i back, after its kernel
+
+    so the input copy of step i+1 and the output copy of step i-1 run while
+    the kernel of step i runs.  The kernels stay in order on one stream: each
+    step stores its new rows before the next step reads the cache.
+
+    Use: fill ``inputs(slot)`` for the slot ``next_slot()`` names, call
+    ``submit()`` (returns a ticket), and ``wait(ticket)`` for the host output
+    of that step.  Before a slot's inputs are filled again, the step that last
+    used it must have been waited for (``submit`` checks this), since its copies
+    read and write that slot's pinned buffers.
+    """
+
+    _ALIGN = 256
+
+    def __init__(self, k_cache, v_cache, num_seqs, num_heads, max_blocks_per_seq, max_context_len, scale,
+                 kv_chunk_size=0, depth=2):
+        if depth < 1:
+            raise ValueError("depth must be >= 1")
+        nb, bs, hkv, d = k_cache.shape
+        dev = k_cache.device
+        B, hq = num_seqs, num_heads
+        self.device, self.depth = dev, depth
+        spec = [("q", (B, hq, d), torch.bfloat16), ("new_k", (B, hkv, d), torch.bfloat16),
+                ("new_v", (B, hkv, d), torch.bfloat16), ("slot_mapping", (B,), torch.int32),
+                ("block_tables", (B, max_blocks_per_seq), torch.int32), ("context_lens", (B,), torch.int32)]
+        offs, o = [], 0
+        for _, shape, dt in spec:
+            n = math.prod(shape) * torch.empty((), dtype=dt).element_size()
+            offs.append((o, n))
+            o = (o + n + self._ALIGN - 1) // self._ALIGN * self._ALIGN
+        self.h2d_bytes = o
+
+        def views(buf):
+            return {name: buf[a:a + n].view(dt).view(shape) for (name, shape, dt), (a, n) in zip(spec, offs)}
+
+        self.host_in = [torch.zeros(o, dtype=torch.uint8).pin_memory() for _ in range(depth)]
+        self.dev_in = [torch.zeros(o, dtype=torch.uint8, device=dev) for _ in range(depth)]
+        self._h = [views(b) for b in self.host_in]
+        self._d = [views(b) for b in self.dev_in]
+        self.dev_out = [torch.empty(B, hq, d, dtype=torch.bfloat16, device=dev) for _ in range(depth)]
+        self.host_out = [torch.empty(B, hq, d, dtype=torch.bfloat16).pin_memory() for _ in range(depth)]
+        self.d2h_bytes = self.host_out[0].numel() * self.host_out[0].element_size()
+        ws = pa.decode_workspace_size(B, hq, hkv, d, max_context_len, bs, kv_chunk_size)
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)   # kernels are serialised
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.max_context_len, self.scale, self.kv_chunk_size = max_context_len, scale, kv_chunk_size
+        for h in self._h:
+            h["slot_mapping"].fill_(-1)            # an unfilled step stores nothing and reads nothing
+            h["block_tables"].fill_(-1)
+        for s in range(depth):
+            self.dev_in[s].copy_(self.host_in[s])
+        self.s_h2d = torch.cuda.Stream(dev)
+        self.s_comp = torch.cuda.Stream(dev)
+        self.s_d2h = torch.cuda.Stream(dev)
+        ev = lambda: [torch.cuda.Event() for _ in range(depth)]   # noqa: E731
+        self.h2d_done, self.comp_done, self.d2h_done = ev(), ev(), ev()
+        self._submitted = 0
+        self._waited = [True] * depth
+        for s in range(depth):                      # eager once: kernel set-up happens outside the capture
+            self._kernel(s)
+        torch.cuda.synchronize(dev)
+        self.graphs = []
+        for s in range(depth):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._kernel(s)
+            self.graphs.append(g)
+
+    def _kernel(self, s):
+        d = self._d[s]
+        pa.store_decode(d["q"], d["new_k"], d["new_v"], d["slot_mapping"], self.k_cache, self.v_cache,
+                        d["block_tables"], d["context_lens"], self.max_context_len, self.scale, out=self.dev_out[s],
+                        workspace=self.workspace, kv_chunk_size=self.kv_chunk_size)
+
+    def next_slot(self):
+        return self._submitted % self.depth
+
+    def inputs(self, slot):
+        """Host views of a slot: q, new_k, new_v, slot_mapping, block_tables, context_lens."""
+        return self._h[slot]
+
+    def submit(self):
+        """Enqueue the next step on the slot ``next_slot()`` names; returns its ticket."""
+        s = self.next_slot()
+        if not self._waited[s]:
+            raise RuntimeError("the previous step on this slot has not been waited for")
+        self._waited[s] = False
+        cur = torch.cuda.current_stream(self.device)
+        self.s_h2d.wait_stream(cur)                 # inputs the caller enqueued on its stream
+        self.s_h2d.wait_event(self.comp_done[s])    # the kernel that last read this slot's device inputs
+        with torch.cuda.stream(self.s_h2d):
+            self.dev_in[s].copy_(self.host_in[s], non_blocking=True)
+            self.h2d_done[s].record(self.s_h2d)
+        self.s_comp.wait_event(self.h2d_done[s])
+        self.s_comp.wait_event(self.d2h_done[s])    # the copy that last read this slot's device output
+        with torch.cuda.stream(self.s_comp):
+            self.graphs[s].replay()
+            self.comp_done[s].record(self.s_comp)
+        self.s_d2h.wait_event(self.comp_done[s])
+        with torch.cuda.stream(self.s_d2h):
+            self.host_out[s].copy_(self.dev_out[s], non_blocking=True)
+            self.d2h_done[s].record(self.s_d2h)
+        self._submitted += 1
+        return self._submitted - 1
+
+    def wait(self, ticket):
+        """Block until step ``ticket`` is back in host memory; returns its output [B, Hq, D] (bf16, pinned),
+        valid until the slot is submitted again."""
+        s = ticket % self.depth
+        self.d2h_done[s].synchronize()
+        self._waited[s] = True
+        return self.host_out[s]
+
+    def join(self, stream=None):
+        """Make ``stream`` (default: the current stream) wait for every submitted step."""
+        stream = stream or torch.cuda.current_stream(self.device)
+        for s in range(self.depth):
+            stream.wait_event(self.d2h_done[s])

@@ -1,17 +1,21 @@
-"""Host checks of the device metadata the kernels trust (``include/pa.h``).
+"""Host checks of the device metadata the kernels are given (``include/pa.h``).
 
-The C ABI cannot read device arrays without synchronising, so two kernels take
-some of their metadata on trust:
+The C ABI cannot read device arrays without synchronising, so the kernels
+check this metadata themselves: a violation is skipped or clamped on the
+device and reported through the device error word, after the launch:
 
-- ``pa_prefill_varlen`` trusts ``cu_seqlens_q/k`` to agree with ``total_q``,
-  ``max_seqlen_q/k`` and the width of the block tables;
+- ``pa_prefill_varlen`` needs ``cu_seqlens_q/k`` to agree with ``total_q``,
+  ``max_seqlen_q/k`` and the width of the block tables (a sequence that does
+  not is skipped, code 8);
 - ``pa_store_decode`` writes the new row at the slot the block table names for
-  position ``L - 1``.
+  position ``L - 1`` (another slot is not written, code 5; a block id outside
+  the cache neither, code 6).
 
-These functions check those preconditions on host copies of the arrays and
-raise ``ValueError`` naming the first violation.  The Python binding runs them
-when a call passes ``validate=True`` (which synchronises); a caller that builds
-its metadata on the host can run them before uploading.
+These functions check the same rules on host copies of the arrays before
+anything is launched and raise ``ValueError`` naming the first violation.  The
+Python binding runs them when a call passes ``validate=True`` (which
+synchronises); a caller that builds its metadata on the host can run them
+before uploading.
 """
 from __future__ import annotations
 

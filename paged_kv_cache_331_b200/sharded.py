@@ -54,20 +54,44 @@ def shard_tables(block_tables: np.ndarray, context_lens: np.ndarray, block_size:
 
 
 class ShardedDecode:
-    """One decode step over a context sharded across the ranks of a process group."""
+    """One decode step over a context sharded across the ranks of a process group.
 
-    def __init__(self, group=None):
-        import torch.distributed as dist
-        self.dist = dist
-        self.group = group
-        self.world = dist.get_world_size(group)
+    ``gather(t)`` returns the ranks' copies of ``t`` stacked along a new leading
+    axis, ``[world, *t.shape]``, rank r's at index r.  By default it is an
+    all-gather over ``group`` (NCCL over NVLink for CUDA tensors, gloo for CPU
+    tensors); a caller may pass its own exchange with the same contract
+    (``world`` is then required).
+    """
+
+    def __init__(self, group=None, *, gather=None, world=None):
+        if gather is None:
+            import torch.distributed as dist
+            self.dist = dist
+            self.group = group
+            self.world = dist.get_world_size(group)
+            self._gather = self._all_gather
+        else:
+            if world is None or world < 1:
+                raise ValueError("an injected gather needs the world size")
+            self.dist, self.group, self.world = None, group, int(world)
+            self._gather = gather
+
+    def _all_gather(self, t):
+        t = t.contiguous()
+        # concatenated along dim 0 (the layout both NCCL and gloo accept), then viewed as [world, *shape]
+        out = torch.empty((self.world * t.shape[0],) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+        self.dist.all_gather_into_tensor(out, t, group=self.group)
+        return out.view((self.world,) + tuple(t.shape))
+
+    def gather(self, t):
+        g = self._gather(t)
+        if tuple(g.shape) != (self.world,) + tuple(t.shape):
+            raise ValueError(f"gather returned shape {tuple(g.shape)}, expected {(self.world,) + tuple(t.shape)}")
+        return g
 
     def __call__(self, q, k_cache, v_cache, local_tables, local_lens, max_local_len, scale, *, out=None,
                  kv_chunk_size=0):
+        """pa_decode_partial over this rank's blocks, the all-gather of (o, lse), then pa_merge_partials."""
         o, lse = pa.decode_partial(q, k_cache, v_cache, local_tables, local_lens, max_local_len, scale,
                                    kv_chunk_size=kv_chunk_size)
-        o_all = torch.empty((self.world,) + tuple(o.shape), dtype=o.dtype, device=o.device)
-        lse_all = torch.empty((self.world,) + tuple(lse.shape), dtype=lse.dtype, device=lse.device)
-        self.dist.all_gather_into_tensor(o_all, o, group=self.group)
-        self.dist.all_gather_into_tensor(lse_all, lse, group=self.group)
-        return pa.merge_partials(o_all, lse_all, out=out)
+        return pa.merge_partials(self.gather(o), self.gather(lse), out=out)

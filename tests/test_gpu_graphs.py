@@ -88,3 +88,54 @@ def test_host_decode_step_matches_the_device_calls(oracle):
     _, f64 = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
     assert_attention_close(out_h, f64, what="host decode step")
     assert pa.device_error() == 0
+
+
+def test_host_decode_pipeline_overlapped_steps_match_sequential_calls(oracle):
+    """Five generation steps through the double-buffered host pipeline: every step appends one token to each
+    sequence (its own q and new K/V row, context one longer), the next step is submitted before the previous
+    one is waited for, and each step's host output must equal the same steps run one by one with
+    pa_store_decode (bitwise) and the oracle's store + decode chain (within tolerance)."""
+    from paged_kv_cache_331_b200.graphs import HostDecodePipeline
+    rng = np.random.default_rng(78)
+    steps = 5
+    final = rng.integers(steps + 1, 3000, 12).astype(np.int32)
+    w = W.decode_workload(final, 16, 8, 128, 256, rng=rng)
+    B = w.num_seqs
+    qs = [W.randn_bf16(rng, w.q.shape) for _ in range(steps)]
+    nks = [W.randn_bf16(rng, w.new_k.shape) for _ in range(steps)]
+    nvs = [W.randn_bf16(rng, w.new_v.shape) for _ in range(steps)]
+    lens = [final - (steps - 1) + k for k in range(steps)]
+    slots = [np.array([W.slots_for_positions(w.block_tables[b], [int(lens[k][b]) - 1], 256)[0] for b in range(B)],
+                      np.int32) for k in range(steps)]
+    a, b = DeviceDecode(w), DeviceDecode(w)
+    pipe = HostDecodePipeline(a.k_cache, a.v_cache, B, 16, w.block_tables.shape[1], 3072, w.scale)
+    bf = lambda arr: torch.from_numpy(np.ascontiguousarray(arr).view(np.int16))   # noqa: E731
+    outs, tickets = [], []
+    for k in range(steps):
+        if k >= pipe.depth:                           # the slot's previous step must have come back
+            outs.append(pipe.wait(tickets[k - pipe.depth]).clone())
+        h = pipe.inputs(pipe.next_slot())
+        h["q"].view(torch.int16).copy_(bf(qs[k]))
+        h["new_k"].view(torch.int16).copy_(bf(nks[k]))
+        h["new_v"].view(torch.int16).copy_(bf(nvs[k]))
+        h["slot_mapping"].copy_(torch.from_numpy(slots[k]))
+        h["block_tables"].copy_(torch.from_numpy(w.block_tables))
+        h["context_lens"].copy_(torch.from_numpy(lens[k]))
+        tickets.append(pipe.submit())
+    for t in tickets[len(outs):]:
+        outs.append(pipe.wait(t).clone())
+    kc, vc = w.k_cache.copy(), w.v_cache.copy()
+    for k in range(steps):
+        dq = torch.from_numpy(qs[k].view(np.int16)).view(torch.bfloat16).cuda()
+        dk = torch.from_numpy(nks[k].view(np.int16)).view(torch.bfloat16).cuda()
+        dv = torch.from_numpy(nvs[k].view(np.int16)).view(torch.bfloat16).cuda()
+        ref = pa.store_decode(dq, dk, dv, torch.from_numpy(slots[k]).cuda(), b.k_cache, b.v_cache, b.block_tables,
+                              torch.from_numpy(lens[k]).cuda(), 3072, w.scale)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[k].view(torch.int16), ref.cpu().view(torch.int16)), f"step {k}"
+        oracle.store_kvcache(nks[k], nvs[k], kc, vc, slots[k])
+        _, f64 = oracle.decode(qs[k], kc, vc, w.block_tables, lens[k], w.scale, want_f64=True)
+        assert_attention_close(outs[k], f64, what=f"pipelined host step {k}")
+    torch.cuda.synchronize()
+    assert torch.equal(a.k_cache.view(torch.int16), b.k_cache.view(torch.int16))
+    assert pa.device_error() == 0

@@ -86,3 +86,30 @@ def test_merge_partials_matches_the_oracle_merge(oracle):
     got = out.float().cpu().numpy()
     assert np.abs(got - ref).max() <= 2 ** -7 * max(1.0, np.abs(ref).max())
     assert (got[2, 3] == 0).all()
+
+
+def test_sharded_decode_call_with_an_injected_gather(oracle):
+    """ShardedDecode.__call__ (partial, exchange, merge) for every emulated rank of 3: the exchange is a gather that
+    puts this rank's partial at its index among the other ranks' partials, computed beforehand, as the all-gather
+    would.  Every rank's output must be the same and match the oracle's unsplit decode."""
+    from paged_kv_cache_331_b200.sharded import ShardedDecode
+    lens, hq, hkv, d, bs, world = [5000, 1, 300, 257], 32, 8, 128, 256, 3
+    rng = np.random.default_rng(91)
+    w = W.decode_workload(np.array(lens, np.int32), hq, hkv, d, bs, rng=rng)
+    dw = DeviceDecode(w)
+    plans = [shard_tables(w.block_tables, w.context_lens, bs, world, r) for r in range(world)]
+    parts = [pa.decode_partial(dw.q, dw.k_cache, dw.v_cache, dev_i32(lt), dev_i32(ll), int(ll.max()), w.scale)
+             for lt, ll in plans]
+    outs = []
+    for r, (lt, ll) in enumerate(plans):
+        def gather(t, r=r):
+            others = [p[0] if t.dim() == 3 else p[1] for p in parts]
+            return torch.stack([t if i == r else others[i] for i in range(world)])
+        sd = ShardedDecode(gather=gather, world=world)
+        outs.append(sd(dw.q, dw.k_cache, dw.v_cache, dev_i32(lt), dev_i32(ll), int(ll.max()), w.scale))
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+    _, ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
+    assert_attention_close(outs[0], ref, what="ShardedDecode over 3 emulated ranks")
+    assert pa.device_error() == 0
