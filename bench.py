@@ -76,13 +76,15 @@ def kernel_source_hash(kind):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kind):
-    """DRAM bytes per launch recorded from an ncu capture, if the kernel source is unchanged since."""
+def profiled_traffic(kind, workload):
+    """DRAM bytes per launch of the kernel on that workload, from an ncu capture summarised under profiles/, if the
+    kernel's sources are unchanged since (same source hash); else None."""
+    want = kernel_source_hash(kind)
     for f in sorted(PROFILES.glob("*.md")) + sorted(PROFILES.glob("*.txt")):
-        text = f.read_text()
-        m = re.search(rf"traffic_per_launch\[{kind}\]\s*=\s*([0-9.eE+]+)\s+source_sha=([0-9a-f]+)", text)
-        if m:
-            return float(m.group(1)) if m.group(2) == kernel_source_hash(kind) else None
+        for m in re.finditer(rf"traffic_per_launch\[{kind}:{re.escape(workload)}\]\s*=\s*([0-9.eE+]+)\s+"
+                             rf"source_sha=([0-9a-f]+)", f.read_text()):
+            if m.group(2) == want:
+                return float(m.group(1))
     return None
 
 
@@ -366,6 +368,7 @@ def bench_decode_leg(name, desc, dev, peaks, reps, warmup):
            "kv_gbs": round(kv / (ms / 1e3) / 1e9, 1), "seqs_per_s": round(w.num_seqs / (ms / 1e3), 1),
            "kv_chunk_size": d.chunk, "launches_per_step": d.launches_per_step,
            "roofline": decode_roofline(d, ms, peaks, "pa_store_decode")}
+    res["roofline"]["traffic"] = profiled_traffic("decode", w.name)
     if name == "tiny_decode":
         res["latency_us"] = round(ms * 1e3, 2)
         res["eager_call_us"] = round(float(np.median(eager)) * 1e3, 2)
@@ -448,7 +451,7 @@ def bench_decode(args, world, rank, dev, peaks):
     value = total_kv / (elapsed_ms / 1e3) / 1e9
     seqs = sum_over_ranks(float(w.num_seqs), world) * K / (elapsed_ms / 1e3)
     roof = decode_roofline(d, decode_ms, peaks, "pa_store_decode (decode_split_kernel: store + decode)")
-    roof["traffic"] = profiled_traffic("decode")
+    roof["traffic"] = profiled_traffic("decode", w.name)
 
     # end to end through host buffers: every step copies q, the new K/V rows and the metadata (one packed pinned
     # buffer) to the device, runs the fused store + decode, and copies out back; the host waits for each step's
@@ -580,7 +583,7 @@ def bench_prefill(args, dev, peaks):
         "l2": "flushed before every rep: a 256 MB buffer written, then another 256 MB read",
         "total_q": int(w.cu_seqlens_q[-1]), "ms": prefill_ms, "flops": flops, "tflops": tflops,
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": tflops / peak_tf, "traffic": profiled_traffic("prefill"),
+                     "frac": tflops / peak_tf, "traffic": profiled_traffic("prefill", w.name),
                      "peak_kind": f"bf16 burst ({peaks.get('source')})"},
         "sustained": sustained,
         "store": {"rows": int(w.cu_seqlens_q[-1]), "ms": store_ms, "gbs": store_gbs,

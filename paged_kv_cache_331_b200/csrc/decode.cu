@@ -47,7 +47,10 @@ constexpr int kThreads = (kWarps + 1) * 32;
 // increment completes the count merges every chunk's partial and puts the
 // counter back to zero for the next launch that uses the slot.  The host
 // rotates slots between launches, so launches in flight at the same time on
-// different streams do not share one.
+// different streams do not share one as long as fewer than kMergeSlots are
+// in flight.  A captured CUDA graph keeps the slot it was captured with: a
+// replay overlapping (on another stream) a launch that drew the same slot is
+// outside the contract.
 constexpr int kMergeSlots = 16;
 constexpr int kMergeCounters = 16384;   // sequences x kv heads per launch; above it a merge kernel runs
 __device__ unsigned int g_decode_merge_cnt[kMergeSlots][kMergeCounters];
@@ -220,34 +223,6 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
 
   if (warp == kWarps) {
     // ------------------------------------------------------------ producer --
-    if (p.slot_mapping && chunk == nchunks - 1) {
-      // Fused store: this CTA is the only reader of position L-1 (its last
-      // tile), so it writes the new token's K/V row of kv head g into the
-      // cache before loading any tile.  The slot must be that position's
-      // (any other slot but -1 is reported and not written) and lie inside
-      // the cache (a table entry past the cache is reported, not followed).
-      const int32_t slot = __ldg(p.slot_mapping + b);
-      const int32_t* btb = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq;
-      const int pos = L - 1;
-      const int64_t expect = static_cast<int64_t>(__ldg(btb + pos / p.block_size)) * p.block_size + pos % p.block_size;
-      const bool inside = slot >= 0 && slot < p.num_slots;
-      if (slot == expect && inside) {
-        constexpr int kLanesPerRow = D / 8;   // 16-byte pieces of one head row
-        if (lane < 2 * kLanesPerRow) {
-          const bool is_v = lane >= kLanesPerRow;
-          const int piece = is_v ? lane - kLanesPerRow : lane;
-          const __nv_bfloat16* src = (is_v ? p.new_v + b * p.new_v_stride : p.new_k + b * p.new_k_stride) +
-                                     static_cast<int64_t>(g) * D + piece * 8;
-          __nv_bfloat16* dst = (is_v ? p.v_cache : p.k_cache) +
-                               (static_cast<int64_t>(slot) * p.num_kv_heads + g) * D + piece * 8;
-          *reinterpret_cast<uint4*>(dst) = ld_nc_v4(src);
-          fence_proxy_async_global();
-        }
-      } else if (slot != -1 && lane == 0) {
-        record_error(p.err, slot == expect ? kErrOutOfCache : kErrBadSlot);
-      }
-      __syncwarp();
-    }
     if (lane == 0) {
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
@@ -285,6 +260,40 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
   }
 
   // -------------------------------------------------------------- consumers --
+  // Fused store: this CTA is the only reader of position L-1 (in its last
+  // tile).  The consumer warp whose tokens include it loads the new token's
+  // K/V row of kv head g into registers, writes it to the cache slot (nothing
+  // in this launch reads that slot from global memory, so the store needs no
+  // ordering), and once the last tile has landed overwrites that row of the
+  // staged tile in shared memory, which its TMA load may have read before
+  // the store.  The slot must be that position's (any other slot but -1 is
+  // reported and not written) and lie inside the cache (a table entry past
+  // the cache is reported, not followed).
+  constexpr int kRowPieces = D / 8;   // 16-byte pieces of one head row
+  int patch_row = -1;                 // row of position L-1 in the last tile, if this warp owns it
+  uint4 new_piece = make_uint4(0, 0, 0, 0);   // lanes < kRowPieces: K piece lane; next kRowPieces: V pieces
+  if (p.slot_mapping && chunk == nchunks - 1) {
+    const int32_t slot = __ldg(p.slot_mapping + b);
+    const int32_t* btb = p.block_tables + static_cast<int64_t>(b) * p.max_blocks_per_seq;
+    const int pos = L - 1;
+    const int64_t expect = static_cast<int64_t>(__ldg(btb + pos / p.block_size)) * p.block_size + pos % p.block_size;
+    if (slot == expect && slot >= 0 && slot < p.num_slots) {
+      const int idx = pos - (start + (ntiles - 1) * kTile);   // position within the last tile
+      if (idx / kTPW == warp) {
+        patch_row = idx;
+        if (lane < 2 * kRowPieces) {
+          const bool is_v = lane >= kRowPieces;
+          const int piece = is_v ? lane - kRowPieces : lane;
+          new_piece = ld_nc_v4((is_v ? p.new_v + b * p.new_v_stride : p.new_k + b * p.new_k_stride) +
+                               static_cast<int64_t>(g) * D + piece * 8);
+          *reinterpret_cast<uint4*>((is_v ? p.v_cache : p.k_cache) +
+                                    (static_cast<int64_t>(slot) * p.num_kv_heads + g) * D + piece * 8) = new_piece;
+        }
+      }
+    } else if (slot != -1 && warp == 0 && lane == 0) {
+      record_error(p.err, slot == expect ? kErrOutOfCache : kErrBadSlot);
+    }
+  }
   const int li = lane & 7, gi = lane >> 3;
   const int hsel = head_of_lane<GP, HB>(li);            // head whose score this lane ends up with
   constexpr int kHeadBits = (7 << (3 - HB)) & 7;
@@ -320,6 +329,15 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
   for (int it = 0; it < ntiles; ++it) {
     const int s = it % kStages;
     if (!mbar_wait(&full[s], (it / kStages) & 1, p.err)) break;
+    if (it == ntiles - 1 && patch_row >= 0) {   // the new row replaces what TMA staged for position L-1
+      if (lane < 2 * kRowPieces) {
+        const bool is_v = lane >= kRowPieces;
+        const int piece = is_v ? lane - kRowPieces : lane;
+        *reinterpret_cast<uint4*>((is_v ? sV : sK) + (static_cast<size_t>(s) * kTile + patch_row) * D + piece * 8) =
+            new_piece;
+      }
+      __syncwarp();
+    }
     const int valid = min(kTile, end - (start + it * kTile));
     const int nw = min(kTPW, valid - wbase);
     if (nw > 0) {
