@@ -218,6 +218,11 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int3
  *                 bytes (may be NULL when that size is 0); fully written
  *                 before it is read, so its contents need no initialisation.
  *                 Concurrent calls must not share a workspace.
+ *                 Calls that overlap on the GPU (other streams) use distinct
+ *                 merge counters while fewer than 16 are in flight; a CUDA
+ *                 graph keeps the counters it was captured with, so its
+ *                 replays must not overlap a launch that drew the same ones
+ *                 (one captured 16 split launches later, or an eager one).
  */
 PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,

@@ -73,7 +73,10 @@ constexpr uint32_t kChunkBytes = kBM * 128;   // one 64-element-wide, 128-row sw
 // pairs {next item, CTAs finished}; CTAs take items with atomicAdd, and the
 // last CTA to finish puts both counters back to zero for the next launch that
 // uses the slot.  The host rotates slots between launches so that launches in
-// flight at the same time (on different streams) do not share one.
+// flight at the same time (on different streams) do not share one, as long as
+// fewer than kSchedSlots are in flight.  A captured CUDA graph keeps the slot
+// it was captured with: a replay overlapping (on another stream) a launch that
+// drew the same slot is outside the contract.
 constexpr int kSchedSlots = 64;
 __device__ unsigned int g_prefill_sched[kSchedSlots][2];
 
