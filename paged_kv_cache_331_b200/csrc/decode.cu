@@ -55,6 +55,22 @@ constexpr int kMergeSlots = 16;
 constexpr int kMergeCounters = 16384;   // sequences x kv heads per launch; above it a merge kernel runs
 __device__ unsigned int g_decode_merge_cnt[kMergeSlots][kMergeCounters];
 
+// Longest sequences first.  CTAs start roughly in the order of their index,
+// and a launch whose last wave holds long sequences ends with most SMs idle.
+// So, for unsplit launches of kOrderMinSeqs..kOrderMaxSeqs sequences and at
+// most kOrderMaxCtas CTAs, the CTA with index 0 sorts the sequences by
+// decreasing tile count and writes, for every other CTA, the
+// sequence its blockIdx.z position stands for, with that sequence's context
+// length: ((uint64)length << 32) | (sequence + 1).  Each CTA waits for its own
+// entry (0 = not yet written), reads it once and puts 0 back, so the array
+// is clean for the next launch that uses the slot; the host rotates
+// kOrderSlots slots between launches, as for the merge counters.
+constexpr int kOrderMinSeqs = 2;
+constexpr int kOrderMaxSeqs = 512;
+constexpr int kOrderMaxCtas = 8192;
+constexpr int kOrderSlots = 16;
+__device__ unsigned long long g_decode_order[kOrderSlots][kOrderMaxCtas];
+
 struct DecodeParams {
   __nv_bfloat16* out;
   const __nv_bfloat16* q;
@@ -86,6 +102,7 @@ struct DecodeParams {
   __nv_bfloat16* v_cache;
   int64_t num_slots;        // num_blocks * block_size: a slot at or past it is outside the cache
   int32_t num_blocks;
+  int32_t order_slot;       // >= 0: longest sequences first, through g_decode_order[order_slot]; -1: index order
 };
 
 // Per-shape configuration.  Two CTAs share an SM whenever their shared memory
@@ -169,10 +186,11 @@ __device__ __forceinline__ int lane_of_head(int h) {
   return li;
 }
 
+// The work of one CTA: chunk blockIdx.x of kv head blockIdx.y of sequence b,
+// whose context_lens entry is L_raw.
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
-    decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                        const DecodeParams p) {
+__device__ __forceinline__ void decode_cta(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p,
+                                           const int b, const int L_raw) {
   using Cfg = DecodeCfg<D, G>;
   constexpr int kStages = Cfg::kStages;
   constexpr int GP = Cfg::GP, HB = Cfg::HB;
@@ -188,9 +206,8 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::bar_off);
   uint64_t* empty = full + kStages;
 
-  const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int chunk = blockIdx.x, g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int L_raw = __ldg(p.context_lens + b);
   const int L = clamp_context(L_raw, p);
   if (L != L_raw && chunk == 0 && g == 0 && threadIdx.x == 0) record_error(p.err, kErrContextLen);
   const int hq0 = g * G;
@@ -519,6 +536,119 @@ __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
   }
 }
 
+// The sequence this CTA works on, as a packed order entry (see g_decode_order).
+template <int D, int G>
+__device__ __forceinline__ unsigned long long decode_order_entry(const DecodeParams& p) {
+  using Cfg = DecodeCfg<D, G>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ unsigned long long s_entry;
+  unsigned long long* entries = g_decode_order[p.order_slot];
+  const int nseq = static_cast<int>(gridDim.z);
+  const int lin = static_cast<int>((blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x);
+  if (lin == 0) {
+    // A counting sort by tile count, descending, in shared memory that the
+    // TMA ring does not use yet.  (The order within a tile count is whatever
+    // the shared-memory atomics give: only this CTA computes it.)
+    constexpr int kPerThread = (kOrderMaxSeqs + kThreads - 1) / kThreads;
+    constexpr int kBins = 1024;
+    int* hist = reinterpret_cast<int*>(smem + Cfg::k_off);
+    int* seq_at = hist + kBins;
+    int* raw_at = seq_at + kOrderMaxSeqs;
+    int shift = 0;   // tile counts past kBins share bins
+    while ((((p.max_context_len + kTile - 1) / kTile) >> shift) >= kBins) ++shift;
+    for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    int bin[kPerThread], raw[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      const int i = threadIdx.x + u * kThreads;
+      bin[u] = -1;
+      if (i < nseq) {
+        raw[u] = __ldg(p.context_lens + i);
+        const int tiles = (clamp_context(raw[u], p) + kTile - 1) / kTile;
+        bin[u] = kBins - 1 - min(tiles >> shift, kBins - 1);   // longest first
+        atomicAdd(&hist[bin[u]], 1);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {   // exclusive prefix sum of the bins, 32 consecutive bins per lane
+      constexpr int kPerLane = kBins / 32;
+      int run = 0;
+      for (int k = 0; k < kPerLane; ++k) run += hist[threadIdx.x * kPerLane + k];
+      int incl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (static_cast<int>(threadIdx.x) >= o) incl += v;
+      }
+      int off = incl - run;
+      for (int k = 0; k < kPerLane; ++k) {
+        const int c = hist[threadIdx.x * kPerLane + k];
+        hist[threadIdx.x * kPerLane + k] = off;
+        off += c;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+      if (bin[u] >= 0) {
+        const int pos = atomicAdd(&hist[bin[u]], 1);
+        seq_at[pos] = threadIdx.x + u * kThreads;
+        raw_at[pos] = raw[u];
+      }
+    }
+    __syncthreads();
+    const int per_seq = static_cast<int>(gridDim.x * gridDim.y);
+    for (int e = threadIdx.x + 1; e < nseq * per_seq; e += kThreads) {
+      const int z = e / per_seq;
+      entries[e] = (static_cast<unsigned long long>(static_cast<unsigned int>(raw_at[z])) << 32) |
+                   static_cast<unsigned int>(seq_at[z] + 1);
+    }
+    if (threadIdx.x == 0)
+      s_entry = (static_cast<unsigned long long>(static_cast<unsigned int>(raw_at[0])) << 32) |
+                static_cast<unsigned int>(seq_at[0] + 1);
+    __syncthreads();   // the sort's shared memory is free again
+    return s_entry;
+  }
+  if (threadIdx.x == 0) {
+    volatile unsigned long long* mine = entries + lin;
+    unsigned long long e = *mine;
+    if (e == 0ull) {   // CTA 0 (resident: the first to be dispatched) has not written it yet
+      const uint64_t t0 = global_timer_ns();
+      while ((e = *mine) == 0ull) {
+        if (global_timer_ns() - t0 > PA_WAIT_LIMIT_NS) {   // never on a working device: fall back to index order
+          record_error(p.err, kErrWaitTimeout);
+          e = (static_cast<unsigned long long>(static_cast<unsigned int>(__ldg(p.context_lens + blockIdx.z))) << 32) |
+              (blockIdx.z + 1u);
+          break;
+        }
+      }
+    }
+    *mine = 0ull;      // read once: clean for the next launch that uses the slot
+    s_entry = e;
+  }
+  __syncthreads();
+  return s_entry;
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const DecodeParams p) {
+  if (p.order_slot >= 0) {
+    const unsigned long long e = decode_order_entry<D, G>(p);
+    const unsigned int seq = static_cast<unsigned int>(e) - 1u;
+    if (seq < gridDim.z) {
+      decode_cta<D, G>(tmK, tmV, p, static_cast<int>(seq), static_cast<int>(static_cast<unsigned int>(e >> 32)));
+    } else {   // an entry no launch of this shape wrote (a launch on this slot was cut short): index order
+      if (threadIdx.x == 0) record_error(p.err, kErrWaitTimeout);
+      decode_cta<D, G>(tmK, tmV, p, static_cast<int>(blockIdx.z), __ldg(p.context_lens + blockIdx.z));
+    }
+  } else {
+    decode_cta<D, G>(tmK, tmV, p, static_cast<int>(blockIdx.z), __ldg(p.context_lens + blockIdx.z));
+  }
+}
+
 // Merge of split-KV partials: one warp per (sequence, query head).
 //   M = max_c m_c,  out = sum_c 2^(m_c - M) acc_c / sum_c 2^(m_c - M) l_c
 template <int D>
@@ -717,6 +847,13 @@ pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.v_cache = static_cast<__nv_bfloat16*>(const_cast<void*>(a.v_cache));
   p.num_slots = static_cast<int64_t>(a.num_blocks) * a.block_size;
   p.num_blocks = a.num_blocks;
+  static std::atomic<uint32_t> order_launches{0};
+  const int64_t ctas = static_cast<int64_t>(a.max_chunks) * a.num_kv_heads * a.num_seqs;
+  // only unsplit launches: there CTAs differ in length as much as the contexts do
+  p.order_slot = (a.max_chunks == 1 && a.num_seqs >= kOrderMinSeqs && a.num_seqs <= kOrderMaxSeqs &&
+                  ctas <= kOrderMaxCtas)
+                     ? static_cast<int32_t>(order_launches.fetch_add(1) % kOrderSlots)
+                     : -1;
   static std::atomic<uint32_t> launches{0};
   const bool fused_merge = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads <= kMergeCounters;
   p.merge_slot = (a.max_chunks > 1 && fused_merge) ? static_cast<int32_t>(launches.fetch_add(1) % kMergeSlots) : -1;

@@ -118,3 +118,98 @@ def test_decode_empty_batch():
     torch.cuda.synchronize()
     assert out.shape == (0, 4, 64) and o.shape == (0, 4, 64) and lse.shape == (0, 4)
     assert pa.device_error() == 0
+
+
+@pytest.mark.parametrize("n", [512, 600])
+def test_decode_many_sequences_in_and_past_the_longest_first_range(oracle, n):
+    """Up to 512 sequences per launch the CTAs take the longest sequences first (the first CTA ranks the context
+    lengths and tells every other CTA its sequence); above that they follow the sequence index.  Both sides of
+    the limit, with ties in length and empty sequences, against the oracle (the fused store included)."""
+    rng = np.random.default_rng(800 + n)
+    lens = rng.integers(0, 300, n).astype(np.int32)
+    lens[::7] = 128                                      # ties
+    lens[::11] = 0                                       # empty sequences
+    w = W.decode_workload(lens, 4, 2, 64, 64, rng=rng)
+    dw = DeviceDecode(w)
+    out = pa.store_decode(dw.q, dw.new_k, dw.new_v, dw.slot_mapping, dw.k_cache, dw.v_cache, dw.block_tables,
+                          dw.context_lens, int(lens.max()), w.scale)
+    torch.cuda.synchronize()
+    oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
+    _, ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
+    assert_attention_close(out, ref, what=f"decode of {n} sequences")
+    assert pa.device_error() == 0
+
+
+def test_decode_at_the_sequence_limit(oracle):
+    """65 535 sequences in one launch (the most the grid's z dimension holds): index-order dispatch, contexts of
+    1..200 tokens over 64-token blocks, split into 64-token chunks so that the separate merge kernel runs (more
+    than 16 384 sequence x kv-head pairs), and unsplit, against the oracle."""
+    n = 65535
+    rng = np.random.default_rng(65535)
+    lens = rng.integers(1, 201, n).astype(np.int32)
+    w = W.decode_workload(lens, 2, 1, 64, 64, rng=rng)
+    dw = DeviceDecode(w)
+    pa.store_kvcache(dw.new_k, dw.new_v, dw.k_cache, dw.v_cache, dw.slot_mapping)
+    out = pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.context_lens, 200, w.scale, kv_chunk_size=64)
+    whole = pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.context_lens, 200, w.scale)
+    torch.cuda.synchronize()
+    oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
+    _, ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
+    assert_attention_close(out, ref, what="decode of 65 535 sequences")
+    assert_attention_close(whole, ref, what="decode of 65 535 sequences, automatic chunk")
+    assert pa.device_error() == 0
+
+
+def test_decode_one_very_long_context(oracle):
+    """One sequence of 524 288 tokens (2 048 blocks of 256): the automatic split cuts it into 1 024 chunks whose
+    partials the last chunk's CTA merges, against the oracle; plus a second, short sequence."""
+    rng = np.random.default_rng(524288)
+    lens = np.array([524288, 5], np.int32)
+    w = W.decode_workload(lens, 8, 1, 128, 256, rng=rng)
+    dw = DeviceDecode(w)
+    chunk = pa.decode_chunk_size(2, 1, int(lens.max()), 256)
+    assert -(-int(lens.max()) // chunk) >= 512
+    out = pa.store_decode(dw.q, dw.new_k, dw.new_v, dw.slot_mapping, dw.k_cache, dw.v_cache, dw.block_tables,
+                          dw.context_lens, int(lens.max()), w.scale)
+    torch.cuda.synchronize()
+    oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
+    _, ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
+    assert_attention_close(out, ref, what="decode of a 524 288-token context")
+    assert pa.device_error() == 0
+
+
+def test_longest_first_order_is_repeatable_and_graph_safe(oracle):
+    """The dispatch order lives in per-slot device entries that every launch leaves clean: many launches in a
+    row (more than the 16 slots), and replays of one captured graph with changing context lengths, all give
+    bitwise the same output as a fresh eager call on the same inputs."""
+    rng = np.random.default_rng(1717)
+    w = W.decode_workload(np.full(96, 900, np.int32), 16, 8, 128, 256, rng=rng)   # tables cover 900 tokens
+    lens = rng.integers(1, 900, 96).astype(np.int32)
+    dw = DeviceDecode(w)
+    dw.context_lens.copy_(torch.from_numpy(lens))
+    chunk = 1024                                   # no split: the launches take the longest sequences first
+    first = pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.context_lens, 900, w.scale,
+                      kv_chunk_size=chunk)
+    for _ in range(40):
+        again = pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.context_lens, 900, w.scale,
+                          kv_chunk_size=chunk)
+    torch.cuda.synchronize()
+    assert torch.equal(first.view(torch.int16), again.view(torch.int16))
+    out = torch.empty_like(dw.q)
+    cl = dw.context_lens.clone()
+    assert pa.decode_workspace_size(96, 16, 8, 128, 900, 256, chunk) == 0
+    pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, cl, 900, w.scale, out=out, kv_chunk_size=chunk)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, cl, 900, w.scale, out=out, kv_chunk_size=chunk)
+    for trial in range(3):
+        new_lens = rng.integers(1, 900, 96).astype(np.int32)
+        cl.copy_(torch.from_numpy(new_lens))
+        g.replay()
+        eager = pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, cl, 900, w.scale, kv_chunk_size=chunk)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), eager.view(torch.int16)), trial
+        _, ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, new_lens, w.scale, want_f64=True)
+        assert_attention_close(out, ref, what=f"graph replay {trial} with new context lengths")
+    assert pa.device_error() == 0
