@@ -58,8 +58,10 @@ __device__ unsigned int g_decode_merge_cnt[kMergeSlots][kMergeCounters];
 // Longest sequences first.  CTAs start roughly in the order of their index,
 // and a launch whose last wave holds long sequences ends with most SMs idle.
 // So, for unsplit launches of kOrderMinSeqs..kOrderMaxSeqs sequences and at
-// most kOrderMaxCtas CTAs, the CTA with index 0 sorts the sequences by
-// decreasing tile count and writes, for every other CTA, the
+// most kOrderMaxCtas CTAs, the CTAs of the first wave (blockIdx.z below
+// order_first) take their sequences in index order and start at once, and
+// CTA 0 sorts the other sequences by decreasing tile count and writes, for
+// every later CTA, the
 // sequence its blockIdx.z position stands for, with that sequence's context
 // length: ((uint64)length << 32) | (sequence + 1).  Each CTA waits for its own
 // entry (0 = not yet written), reads it once and puts 0 back, so the array
@@ -103,6 +105,7 @@ struct DecodeParams {
   int64_t num_slots;        // num_blocks * block_size: a slot at or past it is outside the cache
   int32_t num_blocks;
   int32_t order_slot;       // >= 0: longest sequences first, through g_decode_order[order_slot]; -1: index order
+  int32_t order_first;      // blockIdx.z positions below it (the first wave) take their sequence in index order
 };
 
 // Per-shape configuration.  Two CTAs share an SM whenever their shared memory
@@ -554,6 +557,7 @@ __device__ __forceinline__ unsigned long long decode_order_entry(const DecodePar
     int* hist = reinterpret_cast<int*>(smem + Cfg::k_off);
     int* seq_at = hist + kBins;
     int* raw_at = seq_at + kOrderMaxSeqs;
+    const int first = p.order_first;   // sequences [first, nseq) are sorted into positions [first, nseq)
     int shift = 0;   // tile counts past kBins share bins
     while ((((p.max_context_len + kTile - 1) / kTile) >> shift) >= kBins) ++shift;
     for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0;
@@ -561,7 +565,7 @@ __device__ __forceinline__ unsigned long long decode_order_entry(const DecodePar
     int bin[kPerThread], raw[kPerThread];
 #pragma unroll
     for (int u = 0; u < kPerThread; ++u) {
-      const int i = threadIdx.x + u * kThreads;
+      const int i = first + threadIdx.x + u * kThreads;
       bin[u] = -1;
       if (i < nseq) {
         raw[u] = __ldg(p.context_lens + i);
@@ -593,22 +597,19 @@ __device__ __forceinline__ unsigned long long decode_order_entry(const DecodePar
     for (int u = 0; u < kPerThread; ++u) {
       if (bin[u] >= 0) {
         const int pos = atomicAdd(&hist[bin[u]], 1);
-        seq_at[pos] = threadIdx.x + u * kThreads;
+        seq_at[pos] = first + threadIdx.x + u * kThreads;
         raw_at[pos] = raw[u];
       }
     }
     __syncthreads();
     const int per_seq = static_cast<int>(gridDim.x * gridDim.y);
-    for (int e = threadIdx.x + 1; e < nseq * per_seq; e += kThreads) {
-      const int z = e / per_seq;
+    for (int e = first * per_seq + threadIdx.x; e < nseq * per_seq; e += kThreads) {
+      const int z = e / per_seq - first;
       entries[e] = (static_cast<unsigned long long>(static_cast<unsigned int>(raw_at[z])) << 32) |
                    static_cast<unsigned int>(seq_at[z] + 1);
     }
-    if (threadIdx.x == 0)
-      s_entry = (static_cast<unsigned long long>(static_cast<unsigned int>(raw_at[0])) << 32) |
-                static_cast<unsigned int>(seq_at[0] + 1);
     __syncthreads();   // the sort's shared memory is free again
-    return s_entry;
+    return (static_cast<unsigned long long>(static_cast<unsigned int>(__ldg(p.context_lens))) << 32) | 1u;
   }
   if (threadIdx.x == 0) {
     volatile unsigned long long* mine = entries + lin;
@@ -635,7 +636,8 @@ template <int D, int G>
 __global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const DecodeParams p) {
-  if (p.order_slot >= 0) {
+  if (p.order_slot >= 0 && (blockIdx.z >= static_cast<unsigned>(p.order_first) ||
+                            (blockIdx.x | blockIdx.y | blockIdx.z) == 0)) {
     const unsigned long long e = decode_order_entry<D, G>(p);
     const unsigned int seq = static_cast<unsigned int>(e) - 1u;
     if (seq < gridDim.z) {
@@ -849,9 +851,15 @@ pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.num_blocks = a.num_blocks;
   static std::atomic<uint32_t> order_launches{0};
   const int64_t ctas = static_cast<int64_t>(a.max_chunks) * a.num_kv_heads * a.num_seqs;
-  // only unsplit launches: there CTAs differ in length as much as the contexts do
+  // the sequence positions whose CTAs all start in the first wave (two CTAs
+  // per SM where the shape allows it, as DecodeCfg::kMinBlocks says)
+  const int per_sm = (a.head_dim == 64 || G <= 4) ? 2 : 1;
+  p.order_first = static_cast<int32_t>(static_cast<int64_t>(current_device_info()->sm_count) * per_sm /
+                                       (static_cast<int64_t>(a.num_kv_heads) * a.max_chunks));
+  // only unsplit launches, where CTAs differ in length as much as the contexts do, and only when some
+  // sequences come after the first wave
   p.order_slot = (a.max_chunks == 1 && a.num_seqs >= kOrderMinSeqs && a.num_seqs <= kOrderMaxSeqs &&
-                  ctas <= kOrderMaxCtas)
+                  ctas <= kOrderMaxCtas && p.order_first < a.num_seqs)
                      ? static_cast<int32_t>(order_launches.fetch_add(1) % kOrderSlots)
                      : -1;
   static std::atomic<uint32_t> launches{0};
