@@ -375,7 +375,8 @@ PA_API pa_status pa_prefill_varlen(void* out, const void* q, const void* k_cache
  * the current device (synchronises the given stream).  Kernels set it instead
  * of hanging when a pipeline wait exceeds its time limit (about one second),
  * and pa_rotary_store_kvcache sets it for a position outside its table.
- * Codes: 0 none, 1 a pipeline wait timed out, 2 the wait for in-flight copies
+ * Codes: 0 none, 1 a pipeline wait (or a decode CTA's wait for its place in
+ * the dispatch order) timed out, 2 the wait for in-flight copies
  * at exit timed out, 3 dynamic shared memory misaligned, 4 rotary position
  * out of range, 5 a pa_store_decode slot that is not the new token's,
  * 6 a slot (other than -1) or a used block-table entry outside the cache
