@@ -108,14 +108,25 @@ struct DecodeParams {
   int32_t order_first;      // blockIdx.z positions below it (the first wave) take their sequence in index order
 };
 
-// Per-shape configuration.  Two CTAs share an SM whenever their shared memory
-// and registers fit, so each SM has eight consumer warps to hide latency.
-template <int D, int G>
+// CTAs per SM of a launch.  Unsplit launches at head_dim 128 with up to four
+// query heads per kv head run three (two stages each): the extra consumer
+// warps hide more of the arithmetic's latency.  Split launches keep two CTAs
+// of three stages, which stream their long chunks faster.
+constexpr int decode_ctas_per_sm(int head_dim, int G, int max_chunks) {
+  return head_dim == 64 ? 2 : (G <= 4 ? (max_chunks == 1 ? 3 : 2) : 1);
+}
+
+// Per-shape configuration.  B CTAs share an SM (as many as shared memory and
+// registers allow), so that each SM has 4*B consumer warps to hide latency;
+// decode_ctas_per_sm picks B for a launch.
+template <int D, int G, int B>
 struct DecodeCfg {
   static constexpr int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));   // group padded to a power of two
   static constexpr int HB = GP == 1 ? 0 : (GP == 2 ? 1 : (GP == 4 ? 2 : 3)); // log2(GP)
-  static constexpr int kStages = (D == 64) ? 4 : (G <= 4 ? 3 : 4);
-  static constexpr int kMinBlocks = (D == 64 || G <= 4) ? 2 : 1;
+  static_assert(D == 64 ? B == 2 : (G <= 4 ? (B == 2 || B == 3) : B == 1), "CTAs per SM for this shape");
+  // three CTAs per SM fit only with two stages each
+  static constexpr int kStages = (D == 64) ? 4 : (G <= 4 ? (B == 3 ? 2 : 3) : 4);
+  static constexpr int kMinBlocks = B;
   static constexpr size_t kv_stage_elems = static_cast<size_t>(kTile) * D;
   static constexpr size_t k_off = 0;
   static constexpr size_t v_off = k_off + kStages * kv_stage_elems * 2;
@@ -191,10 +202,10 @@ __device__ __forceinline__ int lane_of_head(int h) {
 
 // The work of one CTA: chunk blockIdx.x of kv head blockIdx.y of sequence b,
 // whose context_lens entry is L_raw.
-template <int D, int G>
+template <int D, int G, int B>
 __device__ __forceinline__ void decode_cta(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p,
                                            const int b, const int L_raw) {
-  using Cfg = DecodeCfg<D, G>;
+  using Cfg = DecodeCfg<D, G, B>;
   constexpr int kStages = Cfg::kStages;
   constexpr int GP = Cfg::GP, HB = Cfg::HB;
   constexpr int DPL = D / 8;    // query/key dims per lane in QK (8 lanes per token)
@@ -540,9 +551,9 @@ __device__ __forceinline__ void decode_cta(const CUtensorMap& tmK, const CUtenso
 }
 
 // The sequence this CTA works on, as a packed order entry (see g_decode_order).
-template <int D, int G>
+template <int D, int G, int B>
 __device__ __forceinline__ unsigned long long decode_order_entry(const DecodeParams& p) {
-  using Cfg = DecodeCfg<D, G>;
+  using Cfg = DecodeCfg<D, G, B>;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ unsigned long long s_entry;
   unsigned long long* entries = g_decode_order[p.order_slot];
@@ -632,22 +643,22 @@ __device__ __forceinline__ unsigned long long decode_order_entry(const DecodePar
   return s_entry;
 }
 
-template <int D, int G>
-__global__ void __launch_bounds__(kThreads, DecodeCfg<D, G>::kMinBlocks)
+template <int D, int G, int B>
+__global__ void __launch_bounds__(kThreads, DecodeCfg<D, G, B>::kMinBlocks)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const DecodeParams p) {
   if (p.order_slot >= 0 && (blockIdx.z >= static_cast<unsigned>(p.order_first) ||
                             (blockIdx.x | blockIdx.y | blockIdx.z) == 0)) {
-    const unsigned long long e = decode_order_entry<D, G>(p);
+    const unsigned long long e = decode_order_entry<D, G, B>(p);
     const unsigned int seq = static_cast<unsigned int>(e) - 1u;
     if (seq < gridDim.z) {
-      decode_cta<D, G>(tmK, tmV, p, static_cast<int>(seq), static_cast<int>(static_cast<unsigned int>(e >> 32)));
+      decode_cta<D, G, B>(tmK, tmV, p, static_cast<int>(seq), static_cast<int>(static_cast<unsigned int>(e >> 32)));
     } else {   // an entry no launch of this shape wrote (a launch on this slot was cut short): index order
       if (threadIdx.x == 0) record_error(p.err, kErrWaitTimeout);
-      decode_cta<D, G>(tmK, tmV, p, static_cast<int>(blockIdx.z), __ldg(p.context_lens + blockIdx.z));
+      decode_cta<D, G, B>(tmK, tmV, p, static_cast<int>(blockIdx.z), __ldg(p.context_lens + blockIdx.z));
     }
   } else {
-    decode_cta<D, G>(tmK, tmV, p, static_cast<int>(blockIdx.z), __ldg(p.context_lens + blockIdx.z));
+    decode_cta<D, G, B>(tmK, tmV, p, static_cast<int>(blockIdx.z), __ldg(p.context_lens + blockIdx.z));
   }
 }
 
@@ -735,14 +746,14 @@ __global__ void __launch_bounds__(128) merge_lse_kernel(__nv_bfloat16* __restric
     *reinterpret_cast<uint32_t*>(dst + c) = pack_bf16x2(o[c] * inv, o[c + 1] * inv);
 }
 
-template <int D, int G>
-pa_status launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, dim3 grid,
+template <int D, int G, int B>
+pa_status launch_cfg(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, dim3 grid,
                        cudaStream_t stream) {
-  using Cfg = DecodeCfg<D, G>;
+  using Cfg = DecodeCfg<D, G, B>;
   static int configured_device = -1;
   const DeviceInfo* di = current_device_info();
   if (configured_device != di->device) {
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, G, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(Cfg::bytes));
     if (e != cudaSuccess) {
       set_last_error("cudaFuncSetAttribute(decode): %s", cudaGetErrorString(e));
@@ -750,13 +761,25 @@ pa_status launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const Dec
     }
     configured_device = di->device;
   }
-  decode_split_kernel<D, G><<<grid, kThreads, Cfg::bytes, stream>>>(tmK, tmV, p);
+  decode_split_kernel<D, G, B><<<grid, kThreads, Cfg::bytes, stream>>>(tmK, tmV, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("decode launch: %s", cudaGetErrorString(e));
     return PA_ERR_CUDA;
   }
   return PA_OK;
+}
+
+// The configuration decode_ctas_per_sm names for this launch.
+template <int D, int G>
+pa_status launch_split(const CUtensorMap& tmK, const CUtensorMap& tmV, const DecodeParams& p, dim3 grid,
+                       cudaStream_t stream) {
+  if constexpr (D == 128 && G <= 4) {
+    return decode_ctas_per_sm(D, G, p.max_chunks) == 3 ? launch_cfg<D, G, 3>(tmK, tmV, p, grid, stream)
+                                                       : launch_cfg<D, G, 2>(tmK, tmV, p, grid, stream);
+  } else {
+    return launch_cfg<D, G, (D == 64 ? 2 : 1)>(tmK, tmV, p, grid, stream);
+  }
 }
 
 template <int D>
@@ -780,7 +803,7 @@ pa_status dispatch_group(int G, const CUtensorMap& tmK, const CUtensorMap& tmV, 
 }  // namespace
 
 int32_t decode_auto_chunk(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len, int sm_count) {
-  // Enough CTAs to fill every CTA slot (two per SM) several times over,
+  // Enough CTAs to fill every CTA slot (two per SM, as split launches run) several times over,
   // without chunks so short that per-CTA set-up dominates.
   constexpr int kMinChunk = 512;
   constexpr int kWavesTarget = 4;
@@ -851,9 +874,9 @@ pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   p.num_blocks = a.num_blocks;
   static std::atomic<uint32_t> order_launches{0};
   const int64_t ctas = static_cast<int64_t>(a.max_chunks) * a.num_kv_heads * a.num_seqs;
-  // the sequence positions whose CTAs all start in the first wave (two CTAs
-  // per SM where the shape allows it, as DecodeCfg::kMinBlocks says)
-  const int per_sm = (a.head_dim == 64 || G <= 4) ? 2 : 1;
+  // the sequence positions whose CTAs all start in the first wave (at the
+  // CTAs per SM that decode_ctas_per_sm gives this launch)
+  const int per_sm = decode_ctas_per_sm(a.head_dim, G, a.max_chunks);
   p.order_first = static_cast<int32_t>(static_cast<int64_t>(current_device_info()->sm_count) * per_sm /
                                        (static_cast<int64_t>(a.num_kv_heads) * a.max_chunks));
   // only unsplit launches, where CTAs differ in length as much as the contexts do, and only when some
