@@ -545,9 +545,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int col0 = j * kBN;
         if (col0 + kBN > full_keys) {   // tile reaches past some row's last visible key
+          const int lim = p_row - col0;   // keys past it are masked in this row
 #pragma unroll
-          for (int e = 0; e < kBN; ++e)
-            if (col0 + e > p_row) xs[e] = -INFINITY;
+          for (int e = 0; e < kBN; ++e) xs[e] = e > lim ? -INFINITY : xs[e];
         }
         float mx8[8];
 #pragma unroll
