@@ -315,6 +315,7 @@ def timed_launches(fn, reps, dev, before=None):
     """Per-call CUDA-event times (ms) of fn on the current stream; `before` runs untimed ahead of each call."""
     import torch
     ev = []
+    hold_gpu()
     for _ in range(reps):
         if before is not None:
             before()
@@ -411,9 +412,10 @@ def bench_decode(args, world, rank, dev, peaks):
     barrier(world)
     torch.cuda.synchronize(dev)
     with clk:
-        # the flush keeps the GPU busy while the host enqueues the first steps, so the timed region holds no
-        # launch gap; it is not part of the region
+        # the flush and a short spin keep the GPU busy while the host enqueues the first steps, so the timed
+        # region holds no launch gap; neither is part of the region
         flush()
+        hold_gpu()
         i0 = clk.mark()
         t0.record()
         for i in range(K):
@@ -427,6 +429,7 @@ def bench_decode(args, world, rank, dev, peaks):
         # over these reps, which run the same HBM-bound kernels at the same clocks
         Ku = max(3, min(K, 200))
         evu = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Ku)]
+        hold_gpu()
         for i in range(Ku):
             evu[i][0].record()
             d.store()
@@ -508,6 +511,14 @@ def bench_decode(args, world, rank, dev, peaks):
     }
 
 
+def hold_gpu(us=500.0):
+    """Enqueue a spin kernel of about `us` microseconds (clock cycles at up to 2 GHz).  Placed just before a timed
+    region, it keeps the GPU busy while the host queues the region's first launches, so that the first timed
+    event does not wait on the host's launch overhead."""
+    import torch
+    torch.cuda._sleep(int(us * 2000))
+
+
 class L2Flush:
     """Flush between timed reps: write a buffer larger than L2 (126 MB), then read another one, so that the
     write-back of the flush's dirty lines happens before the timed region rather than inside it."""
@@ -546,6 +557,7 @@ def bench_prefill(args, dev, peaks):
     torch.cuda.synchronize(dev)
     reps = max(3, min(args.steps, 100))
     st, pf = [], []
+    hold_gpu()
     for _ in range(reps):
         flush()
         a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
