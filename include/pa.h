@@ -223,8 +223,8 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int3
  *                 graph keeps the counters it was captured with, so its
  *                 replays must not overlap a launch that drew the same ones
  *                 (one captured 16 split launches later, or an eager one).
- * Dispatch order: an unsplit launch of 2..512 sequences (at most 8192 CTAs)
- * takes its longest sequences first.  The CTAs of the first wave start in
+ * Dispatch order: a launch of 2..512 sequences (at most 8192 CTAs, split or
+ * not) takes its longest sequences first.  The CTAs of the first wave start in
  * sequence order; CTA 0 sorts the others by context length and passes each
  * later CTA its sequence through a per-device entry array that every launch
  * leaves clean.  Slots of that array rotate like the merge counters, with the

@@ -57,15 +57,16 @@ __device__ unsigned int g_decode_merge_cnt[kMergeSlots][kMergeCounters];
 
 // Longest sequences first.  CTAs start roughly in the order of their index,
 // and a launch whose last wave holds long sequences ends with most SMs idle.
-// So, for unsplit launches of kOrderMinSeqs..kOrderMaxSeqs sequences and at
-// most kOrderMaxCtas CTAs, the CTAs of the first wave (blockIdx.z below
-// order_first) take their sequences in index order and start at once, and
-// CTA 0 sorts the other sequences by decreasing tile count and writes, for
-// every later CTA, the
-// sequence its blockIdx.z position stands for, with that sequence's context
-// length: ((uint64)length << 32) | (sequence + 1).  Each CTA waits for its own
-// entry (0 = not yet written), reads it once and puts 0 back, so the array
-// is clean for the next launch that uses the slot; the host rotates
+// So, for launches of kOrderMinSeqs..kOrderMaxSeqs sequences and at most
+// kOrderMaxCtas CTAs, split or not (the chunks of a long sequence are full,
+// those of a short one few or partial), the CTAs of the first wave
+// (blockIdx.z below order_first) take their sequences in index order and
+// start at once, and CTA 0 sorts the other sequences by decreasing tile count
+// and writes, for every later CTA, the sequence its blockIdx.z position
+// stands for, with that sequence's context length:
+// ((uint64)length << 32) | (sequence + 1).  Each CTA waits for its own entry
+// (0 = not yet written), reads it once and puts 0 back, so the array is
+// clean for the next launch that uses the slot; the host rotates
 // kOrderSlots slots between launches, as for the merge counters.
 constexpr int kOrderMinSeqs = 2;
 constexpr int kOrderMaxSeqs = 512;
@@ -879,9 +880,8 @@ pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int per_sm = decode_ctas_per_sm(a.head_dim, G, a.max_chunks);
   p.order_first = static_cast<int32_t>(static_cast<int64_t>(current_device_info()->sm_count) * per_sm /
                                        (static_cast<int64_t>(a.num_kv_heads) * a.max_chunks));
-  // only unsplit launches, where CTAs differ in length as much as the contexts do, and only when some
-  // sequences come after the first wave
-  p.order_slot = (a.max_chunks == 1 && a.num_seqs >= kOrderMinSeqs && a.num_seqs <= kOrderMaxSeqs &&
+  // only when some sequences come after the first wave
+  p.order_slot = (a.num_seqs >= kOrderMinSeqs && a.num_seqs <= kOrderMaxSeqs &&
                   ctas <= kOrderMaxCtas && p.order_first < a.num_seqs)
                      ? static_cast<int32_t>(order_launches.fetch_add(1) % kOrderSlots)
                      : -1;

@@ -120,11 +120,13 @@ def test_decode_empty_batch():
     assert pa.device_error() == 0
 
 
+@pytest.mark.parametrize("chunk", [0, 128])
 @pytest.mark.parametrize("n", [512, 600])
-def test_decode_many_sequences_in_and_past_the_longest_first_range(oracle, n):
+def test_decode_many_sequences_in_and_past_the_longest_first_range(oracle, n, chunk):
     """Up to 512 sequences per launch the CTAs take the longest sequences first (the first CTA ranks the context
     lengths and tells every other CTA its sequence); above that they follow the sequence index.  Both sides of
-    the limit, with ties in length and empty sequences, against the oracle (the fused store included)."""
+    the limit, with ties in length and empty sequences, unsplit and split into 128-token chunks, against the
+    oracle (the fused store included)."""
     rng = np.random.default_rng(800 + n)
     lens = rng.integers(0, 300, n).astype(np.int32)
     lens[::7] = 128                                      # ties
@@ -132,11 +134,11 @@ def test_decode_many_sequences_in_and_past_the_longest_first_range(oracle, n):
     w = W.decode_workload(lens, 4, 2, 64, 64, rng=rng)
     dw = DeviceDecode(w)
     out = pa.store_decode(dw.q, dw.new_k, dw.new_v, dw.slot_mapping, dw.k_cache, dw.v_cache, dw.block_tables,
-                          dw.context_lens, int(lens.max()), w.scale)
+                          dw.context_lens, int(lens.max()), w.scale, kv_chunk_size=chunk)
     torch.cuda.synchronize()
     oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
     _, ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
-    assert_attention_close(out, ref, what=f"decode of {n} sequences")
+    assert_attention_close(out, ref, what=f"decode of {n} sequences, chunk {chunk}")
     assert pa.device_error() == 0
 
 
@@ -178,16 +180,17 @@ def test_decode_one_very_long_context(oracle):
     assert pa.device_error() == 0
 
 
-def test_longest_first_order_is_repeatable_and_graph_safe(oracle):
+@pytest.mark.parametrize("chunk", [1024, 256])
+def test_longest_first_order_is_repeatable_and_graph_safe(oracle, chunk):
     """The dispatch order lives in per-slot device entries that every launch leaves clean: many launches in a
     row (more than the 16 slots), and replays of one captured graph with changing context lengths, all give
-    bitwise the same output as a fresh eager call on the same inputs."""
+    bitwise the same output as a fresh eager call on the same inputs; unsplit (1024-token chunks) and split
+    into up to four chunks merged in the kernel (256)."""
     rng = np.random.default_rng(1717)
     w = W.decode_workload(np.full(96, 900, np.int32), 16, 8, 128, 256, rng=rng)   # tables cover 900 tokens
     lens = rng.integers(1, 900, 96).astype(np.int32)
     dw = DeviceDecode(w)
     dw.context_lens.copy_(torch.from_numpy(lens))
-    chunk = 1024                                   # no split: the launches take the longest sequences first
     first = pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.context_lens, 900, w.scale,
                       kv_chunk_size=chunk)
     for _ in range(40):
@@ -197,12 +200,16 @@ def test_longest_first_order_is_repeatable_and_graph_safe(oracle):
     assert torch.equal(first.view(torch.int16), again.view(torch.int16))
     out = torch.empty_like(dw.q)
     cl = dw.context_lens.clone()
-    assert pa.decode_workspace_size(96, 16, 8, 128, 900, 256, chunk) == 0
-    pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, cl, 900, w.scale, out=out, kv_chunk_size=chunk)
+    assert (pa.decode_workspace_size(96, 16, 8, 128, 900, 256, chunk) == 0) == (chunk >= 900)
+    ws = torch.empty(max(16, pa.decode_workspace_size(96, 16, 8, 128, 900, 256, chunk)), dtype=torch.uint8,
+                     device=dw.q.device)
+    pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, cl, 900, w.scale, out=out, workspace=ws,
+              kv_chunk_size=chunk)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, cl, 900, w.scale, out=out, kv_chunk_size=chunk)
+        pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, cl, 900, w.scale, out=out, workspace=ws,
+                  kv_chunk_size=chunk)
     for trial in range(3):
         new_lens = rng.integers(1, 900, 96).astype(np.int32)
         cl.copy_(torch.from_numpy(new_lens))
