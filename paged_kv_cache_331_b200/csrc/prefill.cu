@@ -156,8 +156,10 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float
   x1 = fmaxf(x1, -125.f);
   float t0 = kRoundMagic, t1 = kRoundMagic;
   fadd2(t0, t1, x0, x1);                             // t = x + magic (round to nearest integer)
+  float n0 = -kRoundMagic, n1 = -kRoundMagic;
+  fadd2(n0, n1, t0, t1);                             // n = t - magic, exact
   float f0 = x0, f1 = x1;
-  ffma2(f0, f1, t0 - kRoundMagic, t1 - kRoundMagic, -1.f, -1.f);   // f = x - n
+  ffma2(f0, f1, n0, n1, -1.f, -1.f);                 // f = x - n
   float p0 = kExpC2, p1 = kExpC2;
   ffma2(p0, p1, f0, f1, kExpC3, kExpC3);
   float q0 = kExpC1, q1 = kExpC1;
