@@ -516,7 +516,9 @@ def hold_gpu(us=500.0):
     region, it keeps the GPU busy while the host queues the region's first launches, so that the first timed
     event does not wait on the host's launch overhead."""
     import torch
-    torch.cuda._sleep(int(us * 2000))
+    sleep = getattr(torch.cuda, "_sleep", None)   # a spin kernel of N clock cycles
+    if sleep is not None:
+        sleep(int(us * 2000))
 
 
 class L2Flush:
