@@ -174,7 +174,8 @@ PA_API int32_t pa_decode_chunk_size(int32_t num_seqs, int32_t num_kv_heads, int3
  * waves of two CTAs per SM: no split while num_seqs * num_kv_heads already
  * reaches 8 * sm_count or max_context_len <= 512; otherwise the split count
  * within one of that target whose chunks (whole 64-token tiles) overhang the
- * longest context least, and at most ceil(max_context_len / 512) chunks.
+ * longest context least (of equal overhangs, the fewest chunks), and at most
+ * ceil(max_context_len / 512) chunks.
  * Returns -1 for invalid arguments.
  */
 PA_API int32_t pa_decode_chunk_size_for(int32_t num_seqs, int32_t num_kv_heads, int32_t max_context_len,

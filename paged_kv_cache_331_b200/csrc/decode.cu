@@ -817,9 +817,11 @@ int32_t decode_auto_chunk(int32_t num_seqs, int32_t num_kv_heads, int32_t max_co
   splits = splits < 1 ? 1 : (splits > max_splits ? max_splits : splits);
   // Among one split fewer or more, prefer the count whose chunks (whole
   // tiles) cover the longest context with the least overhang: a short last
-  // chunk leaves its CTA idle for most of a wave (ties: more CTAs).
+  // chunk leaves its CTA idle for most of a wave.  Ties go to fewer CTAs:
+  // with the longest sequences dispatched first, fewer merges and CTA
+  // set-ups pay more than the finer balance of smaller chunks.
   int64_t best_chunk = 0, best_waste = INT64_MAX;
-  for (int64_t s2 = splits + 1; s2 >= splits - 1; --s2) {
+  for (int64_t s2 = splits - 1; s2 <= splits + 1; ++s2) {
     if (s2 < 1 || s2 > max_splits) continue;
     const int64_t per = (max_context_len + s2 - 1) / s2;
     const int64_t chunk = ((per + kTile - 1) / kTile) * kTile;
