@@ -880,8 +880,12 @@ pa_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   // the sequence positions whose CTAs all start in the first wave (at the
   // CTAs per SM that decode_ctas_per_sm gives this launch)
   const int per_sm = decode_ctas_per_sm(a.head_dim, G, a.max_chunks);
-  p.order_first = static_cast<int32_t>(static_cast<int64_t>(current_device_info()->sm_count) * per_sm /
-                                       (static_cast<int64_t>(a.num_kv_heads) * a.max_chunks));
+  // At least position 0 keeps its own sequence: CTA 0, which sorts the rest,
+  // works on sequence 0 whatever the order says, so the sorted order must
+  // start at position 1 even when one position's CTAs fill a whole wave.
+  const int64_t wave_positions = static_cast<int64_t>(current_device_info()->sm_count) * per_sm /
+                                 (static_cast<int64_t>(a.num_kv_heads) * a.max_chunks);
+  p.order_first = static_cast<int32_t>(wave_positions > 1 ? wave_positions : 1);
   // only when some sequences come after the first wave
   p.order_slot = (a.num_seqs >= kOrderMinSeqs && a.num_seqs <= kOrderMaxSeqs &&
                   ctas <= kOrderMaxCtas && p.order_first < a.num_seqs)

@@ -180,6 +180,26 @@ def test_decode_one_very_long_context(oracle):
     assert pa.device_error() == 0
 
 
+def test_longest_first_when_one_position_fills_a_wave(oracle):
+    """A split launch whose kv heads x chunks at one sequence position are more CTAs than one wave holds (64
+    chunks x 8 kv heads): the first CTA, which sorts the other sequences, keeps sequence 0 at position 0, and
+    the longest sequence (the second) is placed after it.  Twenty launches in a row, each against the oracle,
+    so that merge counters left behind by one launch would show in the next."""
+    rng = np.random.default_rng(4096)
+    lens = np.array([100, 4096, 3000], np.int32)
+    w = W.decode_workload(lens, 16, 8, 128, 256, rng=rng)
+    dw = DeviceDecode(w)
+    chunk = 64
+    assert -(-int(lens.max()) // chunk) * 8 > 2 * 148
+    _, ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
+    for i in range(20):
+        out = pa.decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.context_lens, int(lens.max()), w.scale,
+                        kv_chunk_size=chunk)
+        torch.cuda.synchronize()
+        assert_attention_close(out, ref, what=f"launch {i}")
+    assert pa.device_error() == 0
+
+
 @pytest.mark.parametrize("chunk", [1024, 256])
 def test_longest_first_order_is_repeatable_and_graph_safe(oracle, chunk):
     """The dispatch order lives in per-slot device entries that every launch leaves clean: many launches in a
