@@ -5,7 +5,7 @@ import torch
 
 import paged_kv_cache_331_b200 as pa
 from paged_kv_cache_331_b200 import workloads as W
-from gpu_helpers import DeviceDecode, assert_attention_close, host_bits
+from gpu_helpers import DeviceDecode, assert_attention_close, dev_bf16, dev_i32, host_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -177,6 +177,41 @@ def test_decode_one_very_long_context(oracle):
     oracle.store_kvcache(w.new_k, w.new_v, w.k_cache, w.v_cache, w.slot_mapping)
     _, ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.context_lens, w.scale, want_f64=True)
     assert_attention_close(out, ref, what="decode of a 524 288-token context")
+    assert pa.device_error() == 0
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_dispatch_order_fuzz(oracle, seed):
+    """Random shapes across the dispatch paths (unsplit or split, first waves of many or of one sequence
+    position, empty sequences, the longest sequence anywhere): three launches in a row, each with the fused
+    store of a fresh row, against the oracle's store + decode chain."""
+    rng = np.random.default_rng(9000 + seed)
+    hkv = int(rng.choice([1, 2, 4, 8]))
+    g = int(rng.choice([1, 2, 4]))
+    d = int(rng.choice([64, 128]))
+    bs = int(rng.choice([16, 64, 256]))
+    n = int(rng.integers(2, 48))
+    lens = rng.integers(0, int(rng.choice([300, 2000, 6000])), n).astype(np.int32)
+    lens[rng.integers(0, n)] = lens.max() + int(rng.integers(1, 200))      # a longest sequence, anywhere
+    chunk = int(rng.choice([0, 64, 128, 512]))
+    w = W.decode_workload(lens + 3, hkv * g, hkv, d, bs, rng=rng)              # room for three new tokens
+    dw = DeviceDecode(w)
+    kc, vc = w.k_cache.copy(), w.v_cache.copy()
+    cur = lens.copy()
+    for step in range(3):
+        cur = cur + 1
+        slots = np.array([W.slots_for_positions(w.block_tables[b], [int(cur[b]) - 1], bs)[0] for b in range(n)],
+                         np.int32)
+        new_k = W.randn_bf16(rng, (n, hkv, d))
+        new_v = W.randn_bf16(rng, (n, hkv, d))
+        cl = torch.from_numpy(cur).to(dw.q.device)
+        out = pa.store_decode(dw.q, dev_bf16(new_k), dev_bf16(new_v), dev_i32(slots), dw.k_cache, dw.v_cache,
+                              dw.block_tables, cl, int(cur.max()), w.scale, kv_chunk_size=chunk)
+        torch.cuda.synchronize()
+        oracle.store_kvcache(new_k, new_v, kc, vc, slots)
+        _, ref = oracle.decode(w.q, kc, vc, w.block_tables, cur, w.scale, want_f64=True)
+        assert_attention_close(out, ref, what=f"seed {seed} step {step} (hkv {hkv}, g {g}, d {d}, bs {bs}, "
+                                              f"n {n}, chunk {chunk})")
     assert pa.device_error() == 0
 
 
