@@ -283,9 +283,11 @@ PA_API pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache
  * elements, as for pa_store_kvcache; slot_mapping: [num_seqs] int32.  Token b
  * is the newest token of sequence b: slot_mapping[b] must be -1 (nothing is
  * stored) or the slot of position context_lens[b]-1 in block_tables[b].  The
- * CTA that reads that position writes the row first, so the result equals
- * the two separate calls.  Any other slot is not written and sets device
- * error code 5.  key/value rows must be 16-byte aligned with strides that are
+ * CTA that reads that position writes the row to the slot and attends over
+ * the new row (not what the slot held before), so the result equals the two
+ * separate calls.  Any other slot is not written and sets device error code
+ * 5; the right slot past the end of the cache sets code 6 and is not
+ * written either.  key/value rows must be 16-byte aligned with strides that are
  * multiples of 8 elements (PA_ERR_UNSUPPORTED otherwise).  Every other
  * argument, the workspace rule and the errors are pa_decode's.
  * The row is written at the slot the block-table entry for position
