@@ -778,7 +778,10 @@ def run_ours(args, world, rank, local):
         del d, flush
         torch.cuda.empty_cache()
         legs = {}
+        only = set(args.legs.split(",")) if args.legs else None
         for name, desc in DECODE_LEGS.items():
+            if only is not None and name not in only:
+                continue
             reps = max(50, min(args.steps, 500)) if name != "tiny_decode" else 200
             legs[name], dl = bench_decode_leg(name, desc, dev, peaks, reps, max(3, args.warmup))
             del dl
@@ -878,6 +881,8 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--legs", default="",
+                    help="comma-separated decode legs to run (default: all of " + ", ".join(DECODE_LEGS) + ")")
     ap.add_argument("--no-legs", action="store_true",
                     help="skip the per-workload decode legs (tiny, Qwen3-shaped, long context) and the row store")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
